@@ -1,0 +1,208 @@
+"""Python binding of libcq: CQ (Cactus-Quants) Hadamard/codebook weight quantisation on B200.
+
+The functions below only marshal arguments to the C ABI declared in ``include/cq.h``;
+every step of quantise / dequantise / dequant-GEMV runs in the CUDA kernels of
+``libcq.so``.  PyTorch supplies device memory and the current CUDA stream.  There is no
+CPU fallback: if ``libcq.so`` is missing or a call fails, an exception is raised.
+
+Layout (page "How CQ2-bit Quantization Contributes to Needle 2's Small Footprint",
+"Per-Group Storage Breakdown"): ``packed`` is uint8 ``[rows, G, 16*b]`` (b = 2 for
+ternary), ``norms`` is float16 ``[rows, G]`` with ``G = ceil(cols / 128)``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcq.so")
+
+TERNARY = 0
+GROUP_SIZE = 128
+CQ_F32, CQ_BF16 = 0, 1
+
+_STATUS = {0: "CQ_OK", 1: "CQ_ERR_INVALID_ARG", 2: "CQ_ERR_UNSUPPORTED", 3: "CQ_ERR_CUDA",
+           4: "CQ_ERR_ALIGNMENT", 5: "CQ_ERR_WORKSPACE"}
+
+# Every symbol include/cq.h declares (checked by the CPU test suite).
+EXPORTS = ("cq_status_string", "cq_version", "cq_codebook", "cq_packed_bytes", "cq_norm_bytes",
+           "cq_quantize", "cq_dequantize", "cq_dequant_gemv", "cq_gemv_workspace_bytes")
+
+
+class CQError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {lib().cq_status_string(status).decode()}")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libcq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libcq.so not built at {LIB_PATH}; run "
+                              "`python -m hadamard_codebook_bit_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, ll, i, sz = ctypes.c_void_p, ctypes.c_longlong, ctypes.c_int, ctypes.c_size_t
+        L.cq_status_string.argtypes = [i]
+        L.cq_status_string.restype = ctypes.c_char_p
+        L.cq_version.restype = i
+        L.cq_codebook.argtypes = [i, i, ctypes.c_ulonglong, P, P]
+        L.cq_packed_bytes.argtypes = [ll, ll, i, i]
+        L.cq_packed_bytes.restype = sz
+        L.cq_norm_bytes.argtypes = [ll, ll, i]
+        L.cq_norm_bytes.restype = sz
+        L.cq_quantize.argtypes = [P, i, ll, ll, i, i, P, P, P, P]
+        L.cq_dequantize.argtypes = [P, P, ll, ll, i, i, P, P, i, P]
+        L.cq_dequant_gemv.argtypes = [P, P, ll, ll, i, i, P, P, i, P, P, sz, P]
+        L.cq_gemv_workspace_bytes.argtypes = [ll, i]
+        L.cq_gemv_workspace_bytes.restype = sz
+        _lib = L
+    return _lib
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise CQError(rc, what)
+
+
+def field_bits(bits: int) -> int:
+    return 2 if bits == TERNARY else bits
+
+
+def levels(bits: int) -> int:
+    return 3 if bits == TERNARY else 1 << bits
+
+
+def codebook(bits: int, group_size: int = GROUP_SIZE, seed: int = 0) -> np.ndarray:
+    """Default Lloyd-Max / ternary codebook, fp32 ascending (host routine, memoised)."""
+    out = np.zeros(16, np.float32)
+    n = ctypes.c_int(0)
+    _check(lib().cq_codebook(bits, group_size, seed, out.ctypes.data_as(ctypes.c_void_p),
+                             ctypes.byref(n)), "cq_codebook")
+    return out[:n.value].copy()
+
+
+def packed_bytes(rows: int, cols: int, bits: int, group_size: int = GROUP_SIZE) -> int:
+    return int(lib().cq_packed_bytes(rows, cols, bits, group_size))
+
+
+def norm_bytes(rows: int, cols: int, group_size: int = GROUP_SIZE) -> int:
+    return int(lib().cq_norm_bytes(rows, cols, group_size))
+
+
+def gemv_workspace_bytes(cols: int, batch: int) -> int:
+    return int(lib().cq_gemv_workspace_bytes(cols, batch))
+
+
+# ------------------------------------------------------------------------------------------
+# torch-facing wrappers (device tensors, current stream)
+# ------------------------------------------------------------------------------------------
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream(device) -> int:
+    torch = _torch()
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _dev_ptr(t, name: str) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _cb_ptr(cb, device) -> int | None:
+    if cb is None:
+        return None
+    torch = _torch()
+    if cb.dtype != torch.float32 or not cb.is_cuda or cb.device != device:
+        raise ValueError("codebook must be a float32 CUDA tensor on the same device")
+    return _dev_ptr(cb, "codebook")
+
+
+def empty_packed(rows: int, cols: int, bits: int, device, group_size: int = GROUP_SIZE):
+    torch = _torch()
+    G = -(-cols // group_size)
+    return (torch.empty((rows, G, group_size * field_bits(bits) // 8), dtype=torch.uint8,
+                        device=device),
+            torch.empty((rows, G), dtype=torch.float16, device=device))
+
+
+def quantize(w, bits: int, group_size: int = GROUP_SIZE, codebook=None, out=None):
+    """cq_quantize on a 2-D bf16/fp32 CUDA tensor -> (packed uint8, norms float16)."""
+    torch = _torch()
+    if w.dim() != 2:
+        raise ValueError("w must be 2-D [rows, cols]")
+    if w.dtype == torch.bfloat16:
+        dt = CQ_BF16
+    elif w.dtype == torch.float32:
+        dt = CQ_F32
+    else:
+        raise ValueError("w must be bfloat16 or float32")
+    rows, cols = w.shape
+    packed, norms = out if out is not None else empty_packed(rows, cols, bits, w.device, group_size)
+    with torch.cuda.device(w.device):
+        _check(lib().cq_quantize(_dev_ptr(w, "w"), dt, rows, cols, bits, group_size,
+                                 _cb_ptr(codebook, w.device), _dev_ptr(packed, "packed"),
+                                 _dev_ptr(norms, "norms"), _stream(w.device)), "cq_quantize")
+    return packed, norms
+
+
+def dequantize(packed, norms, rows: int, cols: int, bits: int, group_size: int = GROUP_SIZE,
+               codebook=None, out_dtype=None, out=None):
+    """cq_dequantize -> W_hat [rows, cols] (bfloat16 by default, or float32)."""
+    torch = _torch()
+    if out is None:
+        out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+        out = torch.empty((rows, cols), dtype=out_dtype, device=packed.device)
+    if out.dtype == torch.bfloat16:
+        dt = CQ_BF16
+    elif out.dtype == torch.float32:
+        dt = CQ_F32
+    else:
+        raise ValueError("out dtype must be bfloat16 or float32")
+    if norms.dtype != torch.float16:
+        raise ValueError("norms must be float16")
+    with torch.cuda.device(packed.device):
+        _check(lib().cq_dequantize(_dev_ptr(packed, "packed"), _dev_ptr(norms, "norms"), rows,
+                                   cols, bits, group_size, _cb_ptr(codebook, packed.device),
+                                   _dev_ptr(out, "out"), dt, _stream(packed.device)),
+               "cq_dequantize")
+    return out
+
+
+def dequant_gemv(packed, norms, rows: int, cols: int, bits: int, x, group_size: int = GROUP_SIZE,
+                 codebook=None, workspace=None, y=None):
+    """cq_dequant_gemv: y [batch, rows] fp32 = W_hat x for x bf16 [batch, cols]."""
+    torch = _torch()
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    if x.dtype != torch.bfloat16:
+        raise ValueError("x must be bfloat16")
+    batch = x.shape[0]
+    if norms.dtype != torch.float16:
+        raise ValueError("norms must be float16")
+    if y is None:
+        y = torch.empty((batch, rows), dtype=torch.float32, device=packed.device)
+    ws_bytes = gemv_workspace_bytes(cols, batch)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=packed.device)
+    with torch.cuda.device(packed.device):
+        _check(lib().cq_dequant_gemv(_dev_ptr(packed, "packed"), _dev_ptr(norms, "norms"), rows,
+                                     cols, bits, group_size, _cb_ptr(codebook, packed.device),
+                                     _dev_ptr(x, "x"), batch, _dev_ptr(y, "y"),
+                                     _dev_ptr(workspace, "workspace"),
+                                     workspace.numel() * workspace.element_size(),
+                                     _stream(packed.device)), "cq_dequant_gemv")
+    return y

@@ -1,0 +1,215 @@
+// cq_api.cu -- the extern "C" entry points of libcq (declared in include/cq.h).
+//
+// Host side only: argument validation (before any launch), the per-device default
+// codebook, and dispatch to the kernel launchers.  Nothing here computes on the data.
+#include <cstdint>
+#include <mutex>
+
+#include "cq_internal.h"
+
+namespace cq {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// Default codebooks live in device memory of every GPU that used them: slot 0 = ternary,
+// 1 = 2-bit, 2 = 3-bit, 3 = 4-bit.  Filled lazily, once per (device, slot).
+__device__ float g_default_codebooks[4][16];
+
+std::mutex g_mu;
+bool g_default_ready[kMaxDevices][4];
+int g_sm_count[kMaxDevices];
+
+int slot_for_bits(int bits) { return bits == CQ_BITS_TERNARY ? 0 : bits - 1; }
+
+int current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    return dev;
+}
+
+// Device pointer of the default codebook for `bits` on the current device, uploading it on
+// first use (synchronous copy).
+cudaError_t default_codebook(int bits, const float** out) {
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    const int slot = slot_for_bits(bits);
+    std::lock_guard<std::mutex> lock(g_mu);
+    void* base = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&base, g_default_codebooks);
+    if (e != cudaSuccess) return e;
+    float* dst = static_cast<float*>(base) + 16 * slot;
+    if (!g_default_ready[dev][slot]) {
+        float host[16] = {0};
+        if (host_codebook(bits, kGroup, 0, host) < 0) return cudaErrorInvalidValue;
+        e = cudaMemcpy(dst, host, sizeof(host), cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) return e;
+        g_default_ready[dev][slot] = true;
+    }
+    *out = dst;
+    return cudaSuccess;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool bits_ok(int bits) { return bits == CQ_BITS_TERNARY || (bits >= 2 && bits <= 4); }
+
+int check_common(long long rows, long long cols, int bits, int group_size) {
+    if (rows < 0 || cols < 0 || !bits_ok(bits)) return CQ_ERR_INVALID_ARG;
+    if (group_size <= 0 || (group_size & (group_size - 1))) return CQ_ERR_INVALID_ARG;
+    if (group_size != kGroup) return CQ_ERR_UNSUPPORTED;
+    // keep every byte offset well inside 64-bit arithmetic
+    if (cols > 0 && rows > (1LL << 40) / cols) return CQ_ERR_INVALID_ARG;
+    return CQ_OK;
+}
+
+Shape make_shape(long long rows, long long cols) {
+    Shape s;
+    s.rows = rows;
+    s.cols = cols;
+    s.groups_per_row = (cols + kGroup - 1) / kGroup;
+    s.total_groups = rows * s.groups_per_row;
+    return s;
+}
+
+int resolve_codebook(int bits, const float* codebook, const float** cb) {
+    if (codebook != nullptr) {
+        if ((reinterpret_cast<uintptr_t>(codebook) & 3u) != 0) return CQ_ERR_ALIGNMENT;
+        *cb = codebook;
+        return CQ_OK;
+    }
+    return default_codebook(bits, cb) == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
+}
+
+}  // namespace
+
+int sm_count() {
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return 148;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (g_sm_count[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        g_sm_count[dev] = n;
+    }
+    return g_sm_count[dev];
+}
+
+}  // namespace cq
+
+extern "C" {
+
+const char* cq_status_string(int status) {
+    switch (status) {
+        case CQ_OK: return "CQ_OK";
+        case CQ_ERR_INVALID_ARG: return "CQ_ERR_INVALID_ARG: invalid argument";
+        case CQ_ERR_UNSUPPORTED: return "CQ_ERR_UNSUPPORTED: valid but not implemented (group_size must be 128)";
+        case CQ_ERR_CUDA: return "CQ_ERR_CUDA: a CUDA call or kernel launch failed";
+        case CQ_ERR_ALIGNMENT: return "CQ_ERR_ALIGNMENT: device pointer not 16-byte aligned";
+        case CQ_ERR_WORKSPACE: return "CQ_ERR_WORKSPACE: workspace missing or too small";
+        default: return "CQ: unknown status";
+    }
+}
+
+int cq_version(void) { return 10000; }
+
+int cq_codebook(int bits, int group_size, unsigned long long seed, float* out_host, int* n_levels) {
+    if (out_host == nullptr || seed > 0xffffffffULL) return CQ_ERR_INVALID_ARG;
+    const int L = cq::host_codebook(bits, group_size, seed, out_host);
+    if (L < 0) return CQ_ERR_INVALID_ARG;
+    if (n_levels) *n_levels = L;
+    return CQ_OK;
+}
+
+size_t cq_packed_bytes(long long rows, long long cols, int bits, int group_size) {
+    const int fb = cq::field_bits_for(bits);
+    if (rows < 0 || cols < 0 || fb < 0 || group_size < 8 || (group_size & (group_size - 1)))
+        return 0;
+    const long long G = (cols + group_size - 1) / group_size;
+    return static_cast<size_t>(rows) * static_cast<size_t>(G) *
+           static_cast<size_t>(group_size * fb / 8);
+}
+
+size_t cq_norm_bytes(long long rows, long long cols, int group_size) {
+    if (rows < 0 || cols < 0 || group_size < 8 || (group_size & (group_size - 1))) return 0;
+    const long long G = (cols + group_size - 1) / group_size;
+    return 2 * static_cast<size_t>(rows) * static_cast<size_t>(G);
+}
+
+int cq_quantize(const void* w, int w_dtype, long long rows, long long cols, int bits,
+                int group_size, const float* codebook, unsigned char* packed_out,
+                unsigned short* norms_out, void* stream) {
+    if (w_dtype != CQ_F32 && w_dtype != CQ_BF16) return CQ_ERR_INVALID_ARG;
+    int rc = cq::check_common(rows, cols, bits, group_size);
+    if (rc != CQ_OK) return rc;
+    if (rows == 0 || cols == 0) return CQ_OK;  // nothing to quantise
+    if (!w || !packed_out || !norms_out) return CQ_ERR_INVALID_ARG;
+    if (!cq::aligned16(w) || !cq::aligned16(packed_out) || !cq::aligned16(norms_out))
+        return CQ_ERR_ALIGNMENT;
+    const float* cb = nullptr;
+    rc = cq::resolve_codebook(bits, codebook, &cb);
+    if (rc != CQ_OK) return rc;
+    const cudaError_t e = cq::launch_quantize(w, w_dtype, cq::make_shape(rows, cols), bits, cb,
+                                              packed_out, norms_out,
+                                              static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
+}
+
+int cq_dequantize(const unsigned char* packed, const unsigned short* norms, long long rows,
+                  long long cols, int bits, int group_size, const float* codebook, void* out,
+                  int out_dtype, void* stream) {
+    if (out_dtype != CQ_F32 && out_dtype != CQ_BF16) return CQ_ERR_INVALID_ARG;
+    int rc = cq::check_common(rows, cols, bits, group_size);
+    if (rc != CQ_OK) return rc;
+    if (rows == 0 || cols == 0) return CQ_OK;  // nothing to write
+    if (!packed || !norms || !out) return CQ_ERR_INVALID_ARG;
+    if (!cq::aligned16(packed) || !cq::aligned16(norms) || !cq::aligned16(out))
+        return CQ_ERR_ALIGNMENT;
+    const float* cb = nullptr;
+    rc = cq::resolve_codebook(bits, codebook, &cb);
+    if (rc != CQ_OK) return rc;
+    const cudaError_t e = cq::launch_dequantize(packed, norms, cq::make_shape(rows, cols), bits,
+                                                cb, out, out_dtype,
+                                                static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
+}
+
+size_t cq_gemv_workspace_bytes(long long cols, int batch) {
+    if (cols < 0 || batch < 1 || batch > 8) return 0;
+    return cq::gemv_workspace_bytes(cols, batch);
+}
+
+int cq_dequant_gemv(const unsigned char* packed, const unsigned short* norms, long long rows,
+                    long long cols, int bits, int group_size, const float* codebook,
+                    const void* x, int batch, float* y, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+    if (batch < 1 || batch > 8) return CQ_ERR_INVALID_ARG;
+    int rc = cq::check_common(rows, cols, bits, group_size);
+    if (rc != CQ_OK) return rc;
+    if (rows == 0) return CQ_OK;  // y is empty
+    if (!y) return CQ_ERR_INVALID_ARG;
+    if (!cq::aligned16(y)) return CQ_ERR_ALIGNMENT;
+    if (cols == 0) {  // empty inner dimension: y = 0
+        const cudaError_t e = cudaMemsetAsync(y, 0, sizeof(float) * static_cast<size_t>(batch) *
+                                                        static_cast<size_t>(rows),
+                                              static_cast<cudaStream_t>(stream));
+        return e == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
+    }
+    if (!packed || !norms || !x) return CQ_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < cq::gemv_workspace_bytes(cols, batch))
+        return CQ_ERR_WORKSPACE;
+    if (!cq::aligned16(packed) || !cq::aligned16(norms) || !cq::aligned16(x) ||
+        !cq::aligned16(y) || !cq::aligned16(workspace))
+        return CQ_ERR_ALIGNMENT;
+    const float* cb = nullptr;
+    rc = cq::resolve_codebook(bits, codebook, &cb);
+    if (rc != CQ_OK) return rc;
+    const cudaError_t e = cq::launch_dequant_gemv(
+        packed, norms, cq::make_shape(rows, cols), bits, cb, static_cast<const uint16_t*>(x),
+        batch, y, workspace, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,42 @@
+// cq_internal.h -- declarations shared by the C-ABI layer and the kernel files of libcq.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "cq.h"
+
+namespace cq {
+
+constexpr int kGroup = 128;
+
+int levels_for_bits(int bits);
+int field_bits_for(int bits);
+int host_codebook(int bits, int group_size, unsigned long long seed, float* out);
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+// Shape of one quantised matrix as the kernels see it.
+struct Shape {
+    long long rows;
+    long long cols;
+    long long groups_per_row;  // G = ceil(cols / 128)
+    long long total_groups;    // rows * G
+};
+
+// Kernel launchers (one per file).  All return cudaSuccess or the launch error.
+cudaError_t launch_quantize(const void* w, int w_dtype, const Shape& s, int bits,
+                            const float* codebook, uint8_t* packed, uint16_t* norms,
+                            cudaStream_t stream);
+cudaError_t launch_dequantize(const uint8_t* packed, const uint16_t* norms, const Shape& s,
+                              int bits, const float* codebook, void* out, int out_dtype,
+                              cudaStream_t stream);
+size_t gemv_workspace_bytes(long long cols, int batch);
+cudaError_t launch_dequant_gemv(const uint8_t* packed, const uint16_t* norms, const Shape& s,
+                                int bits, const float* codebook, const uint16_t* x, int batch,
+                                float* y, void* workspace, cudaStream_t stream);
+
+}  // namespace cq

@@ -1,0 +1,185 @@
+/*
+ * cq.h -- C ABI of libcq: Cactus-Quants (CQ) group-wise Hadamard/codebook weight
+ * quantisation on NVIDIA B200 (sm_100a).
+ *
+ * The method (pages "Cactus Quants CQ2-bit Quantization" and "How CQ2-bit Quantization
+ * Contributes to Needle 2's Small Footprint"): split each row of a weight matrix into
+ * groups of 128 consecutive elements (zero padding the last one), rotate every group by
+ * the orthonormal Sylvester Walsh-Hadamard matrix H (H[i][k] = (-1)^popcount(i&k)/sqrt(128)),
+ * store the group's L2 norm as fp16, map each normalised component to the nearest entry of
+ * a Gaussian Lloyd-Max codebook scaled by 1/sqrt(128), and bit-pack the indices.
+ * Dequantisation multiplies codeword by norm, rotates back (H is its own inverse) and
+ * drops the padding.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *   Shapes    W is row-major [rows, cols]; groups run along cols; G = ceil(cols / 128)
+ *             groups per row.  Only group_size == 128 is implemented (CQ_ERR_UNSUPPORTED
+ *             otherwise), the pages' default.
+ *   bits      CQ_BITS_TERNARY (0, the "1.58-bit" three-level codebook, stored in 2-bit
+ *             fields), 2, 3 or 4.  L = 3, 4, 8 or 16 levels.
+ *   Packed    Group (r, j) owns the 16*b bytes at offset (r*G + j)*16*b, b = field bits
+ *   layout    (2 for ternary).  Index i of the group sits at bits [b*i, b*i + b) of that
+ *             little-endian bitstream (LSB first).  Norms are a separate fp16 [rows, G]
+ *             array (IEEE binary16 bit patterns, round to nearest even).  (Page "How
+ *             CQ2-bit Quantization Contributes to Needle 2's Small Footprint", "Per-Group
+ *             Storage Breakdown" and "Binary Serialization".)
+ *   Codebook  `codebook` is a DEVICE pointer to L fp32 values sorted ascending and already
+ *             scaled by 1/sqrt(128), or NULL for the built-in default (Lloyd-Max seed 0,
+ *             or the ternary constant).  The first call with NULL for a given bit width
+ *             on a device computes that default on the host and copies it to the device
+ *             synchronously; make that first call before any stream capture.
+ *   Memory    The caller allocates and owns every buffer.  The library allocates nothing
+ *             per call.  All device pointers must be 16-byte aligned.
+ *   Streams   `stream` is a cudaStream_t (NULL = legacy default stream).  Compute calls
+ *             are asynchronous: they enqueue kernels and return without synchronising.
+ *   Empty     rows == 0 or cols == 0 is valid: quantise / dequantise do nothing (their
+ *             pointers may then be NULL) and the GEMV writes y = 0 (rows * batch zeros).
+ *   Errors    Arguments are validated on the host before anything is launched; a bad
+ *             argument returns an error and launches nothing.  A failed launch returns
+ *             CQ_ERR_CUDA.  Kernels never trap and never wait: codes beyond the last level
+ *             (ternary code 3) decode as the last level.
+ *   Threads   Calls may come from several host threads; each call uses the device that
+ *             is current on the calling thread.
+ */
+#ifndef CQ_H
+#define CQ_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CQ_OK = 0,
+    CQ_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, bad bits / dtype / batch  */
+    CQ_ERR_UNSUPPORTED = 2, /* valid per the method but not implemented (group_size != 128) */
+    CQ_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed                  */
+    CQ_ERR_ALIGNMENT = 4,   /* a device pointer is not 16-byte aligned                      */
+    CQ_ERR_WORKSPACE = 5    /* workspace missing or smaller than the size the library asks  */
+} cq_status;
+
+typedef enum {
+    CQ_F32 = 0,  /* IEEE binary32 */
+    CQ_BF16 = 1  /* bfloat16 (top half of a binary32), round to nearest even on output */
+} cq_dtype;
+
+#define CQ_BITS_TERNARY 0
+#define CQ_GROUP_SIZE 128
+
+/* Human-readable name of a status code.  Never NULL; static storage. */
+const char* cq_status_string(int status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int cq_version(void);
+
+/*
+ * cq_codebook -- the default codebook for `bits` (host routine, setup only).
+ *
+ * Page "How Quantization Codebooks Are Trained in Cactus Quants": Lloyd-Max (1-D k-means)
+ * on sorted NumPy-legacy RandomState(seed).randn(400000) samples, quantile initialisation
+ * c_k = x[int((k + 0.5)/L * N)], 200 rounds of midpoint boundaries, left-searchsorted
+ * assignment and cell means, sorted; ternary returns the hard-coded [-1.2240064, 0,
+ * 1.2240064] ("Ternary Special Case Handling").  The levels are divided by
+ * sqrt(group_size) in fp64 and rounded to fp32 ("Production Codebook Generation and
+ * Caching").  Results are memoised per (bits, group_size, seed).
+ *
+ *   bits        CQ_BITS_TERNARY, 2, 3 or 4
+ *   group_size  power of two in [8, 4096]
+ *   seed        RandomState seed (the pages' default is 0); ignored for ternary
+ *   out_host    HOST buffer of at least 16 floats; receives L values, ascending
+ *   n_levels    HOST int* receiving L (may be NULL)
+ * Returns CQ_OK or CQ_ERR_INVALID_ARG.  Touches no GPU.
+ */
+int cq_codebook(int bits, int group_size, unsigned long long seed, float* out_host,
+                int* n_levels);
+
+/*
+ * Byte counts of the two stored arrays (page "How CQ2-bit Quantization Contributes to
+ * Needle 2's Small Footprint", "Per-Group Storage Breakdown": b bits per weight for the
+ * index plus one 16-bit norm per group, nothing else).
+ *   cq_packed_bytes = rows * G * group_size * b / 8      (index stream only)
+ *   cq_norm_bytes   = 2 * rows * G
+ * Return 0 for invalid arguments (and for empty shapes).
+ */
+size_t cq_packed_bytes(long long rows, long long cols, int bits, int group_size);
+size_t cq_norm_bytes(long long rows, long long cols, int group_size);
+
+/*
+ * cq_quantize -- quantise W to packed indices and fp16 norms.
+ *
+ * Page "Cactus Quants CQ2-bit Quantization", "The CQ2-bit Implementation Pipeline"
+ * steps 1-4 (pad and reshape, rotate, normalise, nearest-codeword lookup), with the
+ * stored form of page "How CQ2-bit Quantization Contributes to Needle 2's Small
+ * Footprint", "Binary Serialization".  Per group: v zero padded, r = H v, n = ||r||_2,
+ * u = r / n (u = 0 when n = 0), idx_i = the nearest codeword with ties to the lower
+ * index (decided against fp32 midpoints), norm = fp16(n).
+ *
+ *   w           DEVICE [rows, cols] of w_dtype, row-major, contiguous
+ *   w_dtype     CQ_F32 or CQ_BF16
+ *   rows, cols  >= 0
+ *   bits        CQ_BITS_TERNARY, 2, 3 or 4
+ *   group_size  must be 128
+ *   codebook    DEVICE L fp32 ascending, or NULL for the default
+ *   packed_out  DEVICE cq_packed_bytes(rows, cols, bits, 128) bytes, written fully
+ *   norms_out   DEVICE cq_norm_bytes(rows, cols, 128) bytes (fp16 bit patterns)
+ *   stream      cudaStream_t or NULL
+ * Returns CQ_OK after enqueueing, or an error with nothing launched.
+ */
+int cq_quantize(const void* w, int w_dtype, long long rows, long long cols, int bits,
+                int group_size, const float* codebook, unsigned char* packed_out,
+                unsigned short* norms_out, void* stream);
+
+/*
+ * cq_dequantize -- reconstruct W_hat from packed indices and fp16 norms.
+ *
+ * Page "Cactus Quants CQ2-bit Quantization", "The CQ2-bit Implementation Pipeline"
+ * steps 5-6 (inverse rotate, unpad) and page "How Needle 2 Compresses to a Single
+ * Binary", "Stage 3" (the runtime reconstructs the 2-bit tensors on the fly):
+ * w_hat = H (fp32(norm16) * c[idx]) per group, padding columns dropped.
+ *
+ *   packed, norms  DEVICE, as written by cq_quantize
+ *   rows, cols     >= 0, the shape of W
+ *   bits, group_size, codebook   as for cq_quantize
+ *   out            DEVICE [rows, cols] of out_dtype, row-major, contiguous
+ *   out_dtype      CQ_F32 or CQ_BF16 (bf16 rounds the fp32 result to nearest even)
+ */
+int cq_dequantize(const unsigned char* packed, const unsigned short* norms, long long rows,
+                  long long cols, int bits, int group_size, const float* codebook, void* out,
+                  int out_dtype, void* stream);
+
+/*
+ * cq_dequant_gemv -- y = W_hat x without materialising W_hat.
+ *
+ * Because H is symmetric and orthonormal (page "How CQ2-bit Quantization Contributes to
+ * Needle 2's Small Footprint", "Hadamard Rotation"; page "Cactus Quants CQ2-bit
+ * Quantization", "Hadamard Rotation"), each activation group is rotated once,
+ * x~_j = H x_j, and y[b, r] = sum_j fp32(norm16_rj) * <c[idx_rj], x~_bj>, accumulated in
+ * fp32.  The memory-bandwidth motive is page "Performance Differences Between 2-Bit and
+ * 4-Bit Quantization in Needle", "Model Size and Memory Bandwidth".
+ *
+ *   packed, norms  DEVICE, W quantised as [rows, cols] (rows = outputs, cols = inputs)
+ *   rows, cols     >= 0
+ *   bits           CQ_BITS_TERNARY, 2, 3 or 4
+ *   group_size     must be 128
+ *   codebook       DEVICE L fp32 ascending, or NULL for the default
+ *   x              DEVICE bf16 [batch, cols], row-major
+ *   batch          1..8
+ *   y              DEVICE fp32 [batch, rows], row-major, overwritten
+ *   workspace      DEVICE scratch of at least cq_gemv_workspace_bytes(cols, batch) bytes,
+ *                  16-byte aligned; its contents on entry are ignored and on return are
+ *                  unspecified.  Calls that overlap in time must not share a workspace.
+ */
+int cq_dequant_gemv(const unsigned char* packed, const unsigned short* norms, long long rows,
+                    long long cols, int bits, int group_size, const float* codebook,
+                    const void* x, int batch, float* y, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/* Workspace bytes cq_dequant_gemv needs for this cols and batch (0 if invalid or cols == 0). */
+size_t cq_gemv_workspace_bytes(long long cols, int batch);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CQ_H */

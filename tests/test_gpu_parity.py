@@ -1,0 +1,269 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+Every comparison feeds both sides the same bytes: inputs made on the device are copied
+back for the oracle, and dequantise / GEMV parity is measured on the packed arrays the GPU
+produced.  Tolerances are in tests/parity.py.
+"""
+import math
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import hadamard_codebook_bit_b200 as cq  # noqa: E402
+import synth  # noqa: E402
+from synth import workloads as wl  # noqa: E402
+from tests import parity  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from hadamard_codebook_bit_b200 import build
+    build.build()
+    synth.build()
+    torch.cuda.init()
+
+
+@pytest.fixture(scope="module")
+def ora(oracle_lib):
+    return oracle_lib
+
+
+def to_np(t):
+    """Device tensor -> numpy with the oracle's conventions (bf16/fp16 as uint16 bits)."""
+    t = t.detach().contiguous().cpu()
+    if t.dtype in (torch.bfloat16, torch.float16):
+        return t.view(torch.int16).numpy().view(np.uint16)
+    return t.numpy()
+
+
+def dev_tensor(rows, cols, dtype, seed, tid, sigma):
+    t = torch.empty((rows, cols), dtype=dtype, device=DEV)
+    synth.fill_normal_(t, seed, tid, sigma)
+    return t
+
+
+def roundtrip_check(ora, w_dev, bits, what, codebook=None, out_dtypes=("f32", "bf16")):
+    """Quantise on the GPU and check against the oracle; then dequantise the GPU's packed
+    arrays on both sides.  Returns (packed, norms, w_np, flips)."""
+    rows, cols = w_dev.shape
+    cb_dev = None if codebook is None else torch.tensor(codebook, dtype=torch.float32, device=DEV)
+    cb = cq.codebook(bits) if codebook is None else np.asarray(codebook, np.float32)
+    packed, norms = cq.quantize(w_dev, bits, codebook=cb_dev)
+    torch.cuda.synchronize()
+    w_np = to_np(w_dev)
+    o_packed, o_norms, u = ora.quantize(w_np, bits, codebook_=cb, want_u=True)
+    g_packed, g_norms = to_np(packed), to_np(norms)
+    flips = parity.check_indices(g_packed, o_packed, u, bits, cb, what)
+    w64 = w_np.astype(np.float64) if w_np.dtype != np.uint16 else parity.bf16_to_f64(w_np).reshape(rows, cols)
+    parity.check_norms(g_norms, o_norms, parity.group_norms(w64, cols), what)
+    ref = ora.dequantize(g_packed, g_norms, rows, cols, bits, codebook_=cb)
+    if "f32" in out_dtypes:
+        out = cq.dequantize(packed, norms, rows, cols, bits, codebook=cb_dev, out_dtype=torch.float32)
+        parity.check_dequant_f32(to_np(out), ref, cols, what + " f32")
+    if "bf16" in out_dtypes:
+        out = cq.dequantize(packed, norms, rows, cols, bits, codebook=cb_dev, out_dtype=torch.bfloat16)
+        parity.check_dequant_bf16(to_np(out), ref, what + " bf16")
+    return g_packed, g_norms, w64, flips
+
+
+# ------------------------------------------------------------------------------------------
+# the synthetic generator itself
+# ------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_device_generator_matches_host(dtype):
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    for n, off in [(1, 0), (7, 3), (100003, 0), (4096, 12345)]:
+        t = torch.empty(n, dtype=tdt, device=DEV)
+        synth.fill_normal_(t, 9, 4, 0.02, offset=off)
+        host = synth.normal_host((n,), 9, 4, 0.02, dtype, offset=off)
+        assert np.array_equal(to_np(t), host)
+
+
+# ------------------------------------------------------------------------------------------
+# the five workloads
+# ------------------------------------------------------------------------------------------
+
+def test_small_fp32_matrix(ora):
+    w = wl.SMALL_FP32
+    t = w.tensors[0]
+    host = synth.normal_host((t.rows, t.cols), w.seed, t.tensor_id, w.sigma, "f32")
+    w_dev = torch.from_numpy(host).to(DEV)
+    packed, norms, w64, _ = roundtrip_check(ora, w_dev, 2, "small_fp32")
+    assert packed.size == cq.packed_bytes(t.rows, t.cols, 2) == 32768
+    assert norms.size * 2 == cq.norm_bytes(t.rows, t.cols) == 2048
+    deq = ora.dequantize(packed, norms, t.rows, t.cols, 2)
+    rel = float(np.sum((w64 - deq) ** 2) / np.sum(w64 ** 2))
+    assert 0.10 < rel < 0.13  # expected ~0.116 for a group-normalised Gaussian source
+
+
+@pytest.mark.parametrize("bits", [0, 2, 3, 4])
+def test_outlier_sweep(ora, bits):
+    w_np = wl.outlier_sweep_host()
+    w_dev = torch.from_numpy(w_np).to(DEV)
+    roundtrip_check(ora, w_dev, bits, f"outlier bits={bits}", out_dtypes=("f32",))
+
+
+def test_needle_45m_set(ora):
+    w = wl.NEEDLE_45M
+    total_packed = total_norm = 0
+    for t in w.tensors:
+        w_dev = dev_tensor(t.rows, t.cols, torch.bfloat16, w.seed, t.tensor_id, w.sigma)
+        out = ("f32", "bf16") if t.name in ("head", "l0.k") else ("bf16",)
+        packed, norms, _, _ = roundtrip_check(ora, w_dev, 2, f"needle {t.name}", out_dtypes=out)
+        total_packed += packed.size
+        total_norm += norms.size * 2
+    assert (total_packed, total_norm) == (11206656, 700416)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_llama7b_sampled(ora, bits):
+    """Full 7B-scale set on the device, quantised tensor by tensor exactly as the benchmark
+    does; sampled groups from every tensor checked against the oracle, and every group's
+    norm checked against torch's fp32 norm of the input."""
+    w = wl.LLAMA_7B
+    rng = np.random.default_rng(bits)
+    cb = cq.codebook(bits)
+    per_tensor = 256
+    ins, outs_p, outs_n = [], [], []
+    for t in w.tensors:
+        w_dev = dev_tensor(t.rows, t.cols, torch.bfloat16, w.seed, t.tensor_id, w.sigma)
+        packed, norms = cq.quantize(w_dev, bits)
+        # property at full size: stored norm = fp16(||group||) up to fp16 rounding
+        ref = w_dev.float().view(-1, 128).norm(dim=1)
+        got = norms.float().view(-1)
+        assert torch.all((got - ref).abs() <= ref * 2.0 ** -10 + 1e-12), t.name
+        gidx = torch.from_numpy(rng.choice(t.groups, per_tensor, replace=False)).to(DEV)
+        ins.append(to_np(w_dev.view(-1, 128)[gidx]))
+        outs_p.append(to_np(packed.view(t.groups, -1)[gidx]))
+        outs_n.append(to_np(norms.view(-1)[gidx]))
+        del w_dev, packed, norms
+    w_np = np.concatenate(ins)
+    g_packed, g_norms = np.concatenate(outs_p), np.concatenate(outs_n)
+    o_packed, o_norms, u = ora.quantize(w_np, bits, codebook_=cb, want_u=True)
+    parity.check_indices(g_packed, o_packed, u, bits, cb, "llama7b")
+    parity.check_norms(g_norms, o_norms, parity.group_norms(parity.bf16_to_f64(w_np).reshape(-1, 128), 128))
+    # dequantise the sampled groups on both sides from the GPU's packed arrays
+    rows = w_np.shape[0]
+    pk = torch.from_numpy(g_packed).to(DEV)
+    nm = torch.from_numpy(g_norms.view(np.float16)).to(DEV)
+    deq = cq.dequantize(pk, nm, rows, 128, bits, out_dtype=torch.bfloat16)
+    parity.check_dequant_bf16(to_np(deq), ora.dequantize(g_packed, g_norms, rows, 128, bits), "llama7b")
+
+
+@pytest.mark.parametrize("ti", [0, 1])
+@pytest.mark.parametrize("batch", [1, 8])
+def test_gemv_7b_shapes(ora, ti, batch):
+    w = wl.GEMV_7B
+    t = w.tensors[ti]
+    w_dev = dev_tensor(t.rows, t.cols, torch.bfloat16, w.seed, t.tensor_id, w.sigma)
+    packed, norms = cq.quantize(w_dev, 2)
+    x = torch.empty((batch, t.cols), dtype=torch.bfloat16, device=DEV)
+    synth.fill_normal_(x, w.seed, w.extra["x_ids"][ti], w.extra["x_sigma"])
+    y = cq.dequant_gemv(packed, norms, t.rows, t.cols, 2, x)
+    torch.cuda.synchronize()
+    y_ref = ora.dequant_gemv(to_np(packed), to_np(norms), t.rows, t.cols, 2, to_np(x))
+    parity.check_gemv(to_np(y), y_ref, f"gemv {t.name} b={batch}")
+
+
+# ------------------------------------------------------------------------------------------
+# edge cases
+# ------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("cols", [1, 7, 8, 100, 127, 128, 129, 255, 1000, 1001, 4100])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_ragged_columns(ora, cols, dtype):
+    rows = 37
+    w_dev = dev_tensor(rows, cols, dtype, 11, cols, 0.5)
+    for bits in (0, 2, 3, 4):
+        roundtrip_check(ora, w_dev, bits, f"cols={cols} {dtype} bits={bits}")
+
+
+@pytest.mark.parametrize("bits", [0, 2, 3, 4])
+@pytest.mark.parametrize("cols,batch", [(1, 1), (130, 3), (1000, 8), (4096, 2)])
+def test_gemv_all_bits_and_ragged(ora, bits, cols, batch):
+    rows = 45
+    w_dev = dev_tensor(rows, cols, torch.bfloat16, 12, cols, 0.02)
+    packed, norms = cq.quantize(w_dev, bits)
+    x = torch.empty((batch, cols), dtype=torch.bfloat16, device=DEV)
+    synth.fill_normal_(x, 12, 1000 + cols, 1.0)
+    y = cq.dequant_gemv(packed, norms, rows, cols, bits, x)
+    y_ref = ora.dequant_gemv(to_np(packed), to_np(norms), rows, cols, bits, to_np(x))
+    parity.check_gemv(to_np(y), y_ref, f"gemv bits={bits} cols={cols}")
+
+
+def test_zero_and_spike_groups(ora):
+    w = torch.zeros((6, 384), dtype=torch.float32, device=DEV)
+    w[1, 5] = 0.37
+    w[2, 128 + 77] = -2.5
+    w[3, :] = 1.0  # constant rows rotate onto one component
+    w[4, 256:] = -0.001
+    for bits in (0, 2, 3, 4):
+        roundtrip_check(ora, w, bits, f"special bits={bits}")
+
+
+def test_custom_codebook(ora):
+    cb = np.array([-0.2, -0.05, 0.01, 0.15], np.float32)  # asymmetric, caller supplied
+    w_dev = dev_tensor(64, 640, torch.bfloat16, 13, 0, 0.02)
+    roundtrip_check(ora, w_dev, 2, "custom codebook", codebook=cb)
+
+
+def test_unused_ternary_code_decodes_as_top_level(ora):
+    packed = torch.full((3, 2, 32), 0xFF, dtype=torch.uint8, device=DEV)  # every code = 3
+    norms = torch.full((3, 2), 1.5, dtype=torch.float16, device=DEV)
+    out = cq.dequantize(packed, norms, 3, 256, 0, out_dtype=torch.float32)
+    ref = ora.dequantize(to_np(packed), to_np(norms), 3, 256, 0)
+    parity.check_dequant_f32(to_np(out), ref, 256, "ternary code 3")
+
+
+def test_empty_inputs():
+    w = torch.empty((0, 128), dtype=torch.bfloat16, device=DEV)
+    packed, norms = cq.quantize(w, 2)
+    assert packed.numel() == 0 and norms.numel() == 0
+    y = torch.full((2, 5), 7.0, device=DEV)
+    x = torch.empty((2, 0), dtype=torch.bfloat16, device=DEV)
+    p = torch.empty((5, 0, 32), dtype=torch.uint8, device=DEV)
+    n = torch.empty((5, 0), dtype=torch.float16, device=DEV)
+    cq.dequant_gemv(p, n, 5, 0, 2, x, workspace=torch.empty(16, dtype=torch.uint8, device=DEV), y=y)
+    torch.cuda.synchronize()
+    assert torch.all(y == 0)
+
+
+def test_deterministic_and_stream_ordered(ora):
+    w_dev = dev_tensor(300, 4096, torch.bfloat16, 14, 0, 0.02)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        a = cq.quantize(w_dev, 3)
+        b = cq.quantize(w_dev, 3)
+    s.synchronize()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    c = cq.quantize(w_dev, 3)
+    assert torch.equal(a[0], c[0]) and torch.equal(a[1], c[1])
+
+
+def test_more_than_2g_elements_sampled(ora):
+    """A single tensor of 2^31 + 2^20 bf16 elements (offsets beyond int32)."""
+    rows, cols = 16640, 129088  # 2,147,624,...: cols % 128 == 64 -> padded groups too
+    assert rows * cols > 2 ** 31
+    w_dev = dev_tensor(rows, cols, torch.bfloat16, 15, 0, 0.02)
+    packed, norms = cq.quantize(w_dev, 2)
+    out = cq.dequantize(packed, norms, rows, cols, 2, out_dtype=torch.bfloat16)
+    rng = np.random.default_rng(0)
+    sel = np.sort(rng.choice(rows, 6, replace=False))
+    sel[-1] = rows - 1
+    w_np = to_np(w_dev[torch.from_numpy(sel).to(DEV)])
+    o_packed, o_norms, u = ora.quantize(w_np, 2, want_u=True)
+    g_packed = to_np(packed[torch.from_numpy(sel).to(DEV)])
+    g_norms = to_np(norms[torch.from_numpy(sel).to(DEV)])
+    parity.check_indices(g_packed, o_packed, u, 2, cq.codebook(2), "2G")
+    parity.check_norms(g_norms, o_norms, parity.group_norms(parity.bf16_to_f64(w_np), cols))
+    ref = ora.dequantize(g_packed, g_norms, len(sel), cols, 2)
+    parity.check_dequant_bf16(to_np(out[torch.from_numpy(sel).to(DEV)]), ref, "2G deq")

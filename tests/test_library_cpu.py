@@ -1,0 +1,143 @@
+"""CPU-only checks of libcq: it builds, loads, exports what include/cq.h declares, its host
+routines agree with the oracle, and bad arguments are rejected before anything runs."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import hadamard_codebook_bit_b200 as cq
+from hadamard_codebook_bit_b200 import build as cq_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    cq_build.build()
+    return cq.lib()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "cq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(cq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(cq.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    # and the ELF dynamic table lists them as defined functions
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", cq.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    for name in declared_functions():
+        assert re.search(rf"\bT {name}$", out, flags=re.M), name
+
+
+def test_status_strings(L):
+    for s in range(6):
+        assert L.cq_status_string(s).decode().startswith("CQ")
+    assert b"unknown" in L.cq_status_string(99)
+    assert L.cq_version() == 10000
+
+
+@pytest.mark.parametrize("bits", [0, 2, 3, 4])
+@pytest.mark.parametrize("seed", [0, 7])
+def test_library_codebook_equals_oracle(oracle_lib, bits, seed, L):
+    if bits == 0 and seed:
+        pytest.skip("ternary ignores the seed")
+    ours = cq.codebook(bits, 128, seed)
+    ref = oracle_lib.codebook(bits, 128, seed)
+    assert ours.dtype == np.float32
+    assert np.array_equal(ours, ref)
+
+
+def test_codebook_other_group_sizes(oracle_lib, L):
+    for g in (8, 64, 256, 4096):
+        assert np.array_equal(cq.codebook(2, g), oracle_lib.codebook(2, g))
+
+
+def test_codebook_rejects_bad_arguments(L):
+    out = np.zeros(16, np.float32)
+    p = out.ctypes.data_as(ctypes.c_void_p)
+    for bits, g, seed in [(1, 128, 0), (5, 128, 0), (2, 96, 0), (2, 4, 0), (2, 8192, 0),
+                          (2, 128, 2**32)]:
+        assert L.cq_codebook(bits, g, seed, p, None) == 1
+    assert L.cq_codebook(2, 128, 0, None, None) == 1
+
+
+@pytest.mark.parametrize("rows,cols,bits", [(256, 512, 2), (768, 1000, 3), (1, 1, 0),
+                                            (4096, 11008, 4), (3, 129, 2)])
+def test_byte_counts_match_oracle(oracle_lib, rows, cols, bits, L):
+    assert cq.packed_bytes(rows, cols, bits) == oracle_lib.packed_bytes(rows, cols, bits)
+    assert cq.norm_bytes(rows, cols) == oracle_lib.norm_bytes(rows, cols)
+
+
+def test_byte_counts_edge_cases(L):
+    assert cq.packed_bytes(0, 5, 2) == 0 and cq.norm_bytes(5, 0) == 0
+    assert cq.packed_bytes(-1, 5, 2) == 0 and cq.packed_bytes(5, 5, 7) == 0
+    assert cq.gemv_workspace_bytes(4096, 1) == 32 * 128 * 4
+    assert cq.gemv_workspace_bytes(11008, 8) == 8 * 86 * 128 * 4
+    assert cq.gemv_workspace_bytes(4096, 9) == 0 and cq.gemv_workspace_bytes(4096, 0) == 0
+
+
+# ------------------------------------------------------------------------------------------
+# argument validation: every call below must fail on the host, before any CUDA call
+# ------------------------------------------------------------------------------------------
+
+A = 4096  # a fake, 16-byte aligned "device address": never dereferenced, nothing launches
+
+
+def test_quantize_rejects(L):
+    q = L.cq_quantize
+    assert q(A, 2, 4, 128, 2, 128, None, A, A, None) == 1      # bad dtype
+    assert q(A, 1, -1, 128, 2, 128, None, A, A, None) == 1     # negative rows
+    assert q(A, 1, 4, 128, 1, 128, None, A, A, None) == 1      # bits 1
+    assert q(A, 1, 4, 128, 5, 128, None, A, A, None) == 1      # bits 5
+    assert q(A, 1, 4, 128, 2, 100, None, A, A, None) == 1      # group not a power of two
+    assert q(A, 1, 4, 128, 2, 64, None, A, A, None) == 2       # valid but unsupported
+    assert q(None, 1, 4, 128, 2, 128, None, A, A, None) == 1   # null input
+    assert q(A, 1, 4, 128, 2, 128, None, None, A, None) == 1   # null packed
+    assert q(A + 8, 1, 4, 128, 2, 128, None, A, A, None) == 4  # misaligned
+    assert q(A, 1, 4, 128, 2, 128, None, A, A + 2, None) == 4
+    assert q(A, 1, 1 << 40, 1 << 20, 2, 128, None, A, A, None) == 1  # absurd size
+
+
+def test_empty_shapes_are_no_ops(L):
+    assert L.cq_quantize(None, 1, 0, 128, 2, 128, None, None, None, None) == 0
+    assert L.cq_quantize(None, 0, 7, 0, 4, 128, None, None, None, None) == 0
+    assert L.cq_dequantize(None, None, 0, 64, 3, 128, None, None, 1, None) == 0
+    assert L.cq_dequant_gemv(None, None, 0, 64, 2, 128, None, None, 1, None, None, 0, None) == 0
+
+
+def test_dequantize_rejects(L):
+    d = L.cq_dequantize
+    assert d(A, A, 4, 128, 2, 128, None, A, 3, None) == 1       # bad out dtype
+    assert d(A, A, 4, 128, 6, 128, None, A, 1, None) == 1
+    assert d(A, A, 4, 128, 2, 256, None, A, 1, None) == 2
+    assert d(A, None, 4, 128, 2, 128, None, A, 1, None) == 1
+    assert d(A, A, 4, 128, 2, 128, None, A + 4, 1, None) == 4
+
+
+def test_gemv_rejects(L):
+    g = L.cq_dequant_gemv
+    ws = cq.gemv_workspace_bytes(256, 1)
+    assert g(A, A, 4, 256, 2, 128, None, A, 0, A, A, ws, None) == 1    # batch 0
+    assert g(A, A, 4, 256, 2, 128, None, A, 9, A, A, ws, None) == 1    # batch 9
+    assert g(A, A, 4, 256, 2, 128, None, None, 1, A, A, ws, None) == 1  # null x
+    assert g(A, A, 4, 256, 2, 128, None, A, 1, A, None, ws, None) == 5  # no workspace
+    assert g(A, A, 4, 256, 2, 128, None, A, 1, A, A, ws - 1, None) == 5
+    assert g(A, A, 4, 256, 2, 128, None, A, 1, A + 4, A, ws, None) == 4
+    assert g(A, A, 4, 256, 2, 32, None, A, 1, A, A, ws, None) == 2
+
+
+def test_binding_refuses_cpu_tensors(L):
+    torch = pytest.importorskip("torch")
+    with pytest.raises(ValueError):
+        cq.quantize(torch.zeros(4, 128, dtype=torch.bfloat16), 2)
