@@ -1,0 +1,636 @@
+#!/usr/bin/env python
+"""Benchmark: CQ quantise -> dequantise -> dequant-GEMV over a 7B-scale weight set on B200.
+
+One step is one pass of the whole hot path over the synthetic Llama-shaped bf16 weight set
+(32 layers of q/k/v/o 4096x4096, gate/up 11008x4096, down 4096x11008; 6,476,005,376
+weights, N(0, 0.02^2), seed 3): 2-bit cq_quantize of every tensor, cq_dequantize of every
+tensor back to bf16, and a batch-1 cq_dequant_gemv through every tensor.  Inputs are far
+larger than L2 (13 GB), so no flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cq|reference]
+
+`value` is Gweights/s through the step (all ranks; weak scaling: each rank runs its own
+replica of the set).  Per-op times, 4-bit quantise / dequantise and the GEMV-only
+workload (the two MLP shapes over 48 distinct replicas, batch 1 and 8) are reported in
+`breakdown`.  `--impl reference` times the CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "CQ quant/dequant Gweights/s & % HBM roofline; dequant-GEMV GB/s (1 B200)"
+UNIT = "Gweights/s"
+FALLBACK_HBM_GBS = 6650.0
+
+BITS = 2
+FIELD = {0: 2, 2: 2, 3: 3, 4: 4}
+
+
+def bytes_per_weight_quant(bits: int, in_bytes: int = 2) -> float:
+    """Algorithmic HBM bytes per weight: read the input, write b/8 index bytes + 2/128 norm."""
+    return in_bytes + FIELD[bits] / 8 + 2 / 128
+
+
+def bytes_per_weight_gemv(bits: int) -> float:
+    return FIELD[bits] / 8 + 2 / 128
+
+
+# ------------------------------------------------------------------------------------------
+# distributed plumbing (also exercised by the CPU gloo tests)
+# ------------------------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def replica_tensor_offset(rank: int, n_tensors: int) -> int:
+    """Each rank quantises its own replica of the weight set: tensor ids are offset per rank
+    so replicas hold different data (no data is exchanged between ranks)."""
+    return rank * n_tensors
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# ------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ------------------------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.reader.join(timeout=5)
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != 6:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[2:]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def nvsmi_id(device) -> str:
+    """nvidia-smi --id for a torch device (its UUID, robust to CUDA_VISIBLE_DEVICES)."""
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(device).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except (AttributeError, RuntimeError):
+        return str(device.index or 0)
+
+
+def measured_peak_gbs():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------------------------------
+# the CUDA arm
+# ------------------------------------------------------------------------------------------
+
+class WeightSet:
+    """One replica of the 7B-scale set in a single bf16 buffer, plus per-tensor views of the
+    packed / norm / dequantised / GEMV buffers."""
+
+    def __init__(self, workload, device, id_offset: int, bits: int):
+        import torch
+        import synth
+        self.wl = workload
+        self.bits = bits
+        self.n = workload.numel
+        self.groups = workload.groups
+        blk = 16 * FIELD[bits]
+        self.w = torch.empty(self.n, dtype=torch.bfloat16, device=device)
+        self.packed = torch.empty(self.groups * blk, dtype=torch.uint8, device=device)
+        self.norms = torch.empty(self.groups, dtype=torch.float16, device=device)
+        self.out = torch.empty(self.n, dtype=torch.bfloat16, device=device)
+        self.tensors = []
+        off = goff = 0
+        for t in workload.tensors:
+            v = self.w[off:off + t.numel].view(t.rows, t.cols)
+            synth.fill_normal_(v, workload.seed, t.tensor_id + id_offset, workload.sigma)
+            G = -(-t.cols // 128)
+            self.tensors.append(dict(
+                t=t, w=v,
+                packed=self.packed[goff * blk:(goff + t.groups) * blk].view(t.rows, G, blk),
+                norms=self.norms[goff:goff + t.groups].view(t.rows, G),
+                out=self.out[off:off + t.numel].view(t.rows, t.cols)))
+            off += t.numel
+            goff += t.groups
+        # batch-1 activations, one per input width, and one output vector per tensor
+        self.x = {}
+        for c in sorted({t.cols for t in workload.tensors}):
+            x = torch.empty((1, c), dtype=torch.bfloat16, device=device)
+            synth.fill_normal_(x, workload.seed, 100000 + c + id_offset, 1.0)
+            self.x[c] = x
+        self.y = torch.empty(sum(t.rows for t in workload.tensors), dtype=torch.float32, device=device)
+        yo = 0
+        for d in self.tensors:
+            d["y"] = self.y[yo:yo + d["t"].rows].view(1, -1)
+            yo += d["t"].rows
+        import hadamard_codebook_bit_b200 as cq
+        self.ws = torch.empty(max(cq.gemv_workspace_bytes(c, 1) for c in self.x), dtype=torch.uint8,
+                              device=device)
+
+    def quantize_all(self):
+        import hadamard_codebook_bit_b200 as cq
+        for d in self.tensors:
+            cq.quantize(d["w"], self.bits, out=(d["packed"], d["norms"]))
+
+    def dequantize_all(self):
+        import hadamard_codebook_bit_b200 as cq
+        for d in self.tensors:
+            t = d["t"]
+            cq.dequantize(d["packed"], d["norms"], t.rows, t.cols, self.bits, out=d["out"])
+
+    def gemv_all(self):
+        import hadamard_codebook_bit_b200 as cq
+        for d in self.tensors:
+            t = d["t"]
+            cq.dequant_gemv(d["packed"], d["norms"], t.rows, t.cols, self.bits, self.x[t.cols],
+                            workspace=self.ws, y=d["y"])
+
+    def launches_per_step(self) -> int:
+        return len(self.tensors) * 4  # quantise, dequantise, rotate-x, GEMV
+
+    def capture(self):
+        """Capture each phase's per-tensor calls in a CUDA graph (one replay per phase), so
+        the host's per-call overhead stays off the GPU timeline."""
+        import torch
+        self.graphs = []
+        for fn in (self.quantize_all, self.dequantize_all, self.gemv_all):
+            fn()  # first calls upload the default codebook (must precede capture)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            self.graphs.append(g)
+        return self.graphs
+
+    def release(self):
+        self.graphs = []
+
+
+def time_phases(ws, steps: int, device):
+    """Run `steps` steps, recording events between the phases; returns per-phase ms lists
+    and the total (first start to last end) in ms."""
+    import torch
+    evs = []
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    gq, gd, gg = ws.graphs
+    for _ in range(steps):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        e[0].record()
+        gq.replay()
+        e[1].record()
+        gd.replay()
+        e[2].record()
+        gg.replay()
+        e[3].record()
+        evs.append(e)
+    end.record()
+    torch.cuda.synchronize(device)
+    q = [e[0].elapsed_time(e[1]) for e in evs]
+    d = [e[1].elapsed_time(e[2]) for e in evs]
+    g = [e[2].elapsed_time(e[3]) for e in evs]
+    return q, d, g, start.elapsed_time(end)
+
+
+def time_fn(fn, iters: int, device, warm: int = 2):
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize(device)
+    ts = []
+    for _ in range(iters):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize(device)
+        ts.append(a.elapsed_time(b))
+    return ts
+
+
+def gemv_replica_workload(device, peak):
+    """The two MLP shapes, 2-bit, over 48 distinct quantised replicas (about 575 MB, far more
+    than L2) called round-robin; per-call time = total / 48."""
+    import torch
+    import hadamard_codebook_bit_b200 as cq
+    import synth
+    from synth import workloads as wlm
+    W = wlm.GEMV_7B
+    reps = 48
+    out = {}
+    for ti, t in enumerate(W.tensors):
+        w = torch.empty((t.rows, t.cols), dtype=torch.bfloat16, device=device)
+        synth.fill_normal_(w, W.seed, t.tensor_id, W.sigma)
+        pk, nm = cq.quantize(w, 2)
+        del w
+        pks = [pk.clone() for _ in range(reps)]
+        nms = [nm.clone() for _ in range(reps)]
+        for batch in W.extra["batches"]:
+            x = torch.empty((batch, t.cols), dtype=torch.bfloat16, device=device)
+            synth.fill_normal_(x, W.seed, W.extra["x_ids"][ti], W.extra["x_sigma"])
+            y = torch.empty((batch, t.rows), dtype=torch.float32, device=device)
+            ws = torch.empty(cq.gemv_workspace_bytes(t.cols, batch), dtype=torch.uint8, device=device)
+
+            def run():
+                for i in range(reps):
+                    cq.dequant_gemv(pks[i], nms[i], t.rows, t.cols, 2, x, workspace=ws, y=y)
+
+            run()
+            torch.cuda.synchronize(device)
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                run()
+            ts = time_fn(graph.replay, 5, device)
+            del graph
+            us = statistics.median(ts) / reps * 1000
+            byts = t.groups * (32 + 2) + 2 * t.cols * batch + 4 * t.rows * batch
+            gbs = byts / us / 1e3
+            out[f"{t.rows}x{t.cols}_b{batch}"] = {"us_per_call": round(us, 3), "GB_s": round(gbs, 1),
+                                                  "frac_hbm": round(gbs / peak, 4)}
+        del pks, nms
+    return out
+
+
+def cpu_oracle_sample(target_s: float, threads: int = 0, max_rows: int = 4096):
+    """Time the oracle on rows of layer 0's q tensor (4096 columns): 2-bit quantise,
+    dequantise and a batch-1 GEMV, the same step as the GPU's.  The sample is the first
+    `rows` rows, passed through the oracle repeatedly until about `target_s` seconds have
+    elapsed.  Returns (Gweights/s, rows, passes, seconds, threads)."""
+    import oracle
+    import synth
+    from synth import workloads as wlm
+    W = wlm.LLAMA_7B
+    t0 = W.tensors[0]
+    cols = t0.cols
+    x = synth.normal_host((1, cols), W.seed, 100000 + cols, 1.0, "bf16")
+    nth = threads or oracle.default_threads()
+    rows = 64
+    w = synth.normal_host((rows, cols), W.seed, t0.tensor_id, W.sigma, "bf16")
+
+    def one(wm, r):
+        p, n = oracle.quantize(wm, BITS, nthreads=nth)
+        oracle.dequantize(p, n, r, cols, BITS, nthreads=nth)
+        oracle.dequant_gemv(p, n, r, cols, BITS, x, nthreads=nth)
+
+    s = time.perf_counter()
+    one(w, rows)
+    dt = time.perf_counter() - s
+    rows = int(max(64, min(max_rows, rows * 0.5 * target_s / max(dt, 1e-4))))
+    w = synth.normal_host((rows, cols), W.seed, t0.tensor_id, W.sigma, "bf16")
+    passes = 0
+    s = time.perf_counter()
+    while True:
+        one(w, rows)
+        passes += 1
+        dt = time.perf_counter() - s
+        if dt >= target_s:
+            break
+    return rows * cols * passes / dt / 1e9, rows, passes, dt, nth
+
+
+def run_cuda_arm(args):
+    import torch
+    world, rank, local = dist_env()
+    device = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(device)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=device)
+    import hadamard_codebook_bit_b200 as cq
+    from synth import workloads as wlm
+    cq.lib()
+    W = wlm.LLAMA_7B
+    peak, peak_kind = measured_peak_gbs()
+
+    ws = WeightSet(W, device, replica_tensor_offset(rank, len(W.tensors)), BITS)
+    torch.cuda.synchronize(device)
+    ws.capture()
+    for _ in range(args.warmup):
+        for g in ws.graphs:
+            g.replay()
+    torch.cuda.synchronize(device)
+    barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(nvsmi_id(device)) as clk:
+        q_ms, d_ms, g_ms, total_ms = time_phases(ws, args.steps, device)
+    torch.cuda.synchronize(device)
+    barrier()
+    total_ms = max_over_ranks(total_ms, device)
+    clocks = clk.summary()
+
+    n = W.numel
+    ms_step = total_ms / args.steps
+    value = world * n * args.steps / (total_ms / 1e3) / 1e9
+    qm, dm, gm = (statistics.median(x) for x in (q_ms, d_ms, g_ms))
+    qb = n * bytes_per_weight_quant(BITS)
+    gb = n * bytes_per_weight_gemv(BITS)
+    ops = {
+        "quantize": {"ms": round(qm, 4), "Gweights_s": round(n / qm / 1e6, 1),
+                     "GB_s": round(qb / qm / 1e6, 1), "frac_hbm": round(qb / qm / 1e6 / peak, 4)},
+        "dequantize": {"ms": round(dm, 4), "Gweights_s": round(n / dm / 1e6, 1),
+                       "GB_s": round(qb / dm / 1e6, 1), "frac_hbm": round(qb / dm / 1e6 / peak, 4)},
+        "dequant_gemv": {"ms": round(gm, 4), "Gweights_s": round(n / gm / 1e6, 1),
+                         "GB_s": round(gb / gm / 1e6, 1), "frac_hbm": round(gb / gm / 1e6 / peak, 4)},
+    }
+    dom = "quantize" if qm >= dm else "dequantize"
+    dom_ms = max(qm, dm)
+    achieved = qb / dom_ms / 1e6
+    traffic = load_traffic(dom, n)
+
+    breakdown = {"ops_2bit": ops}
+    if not args.quick:
+        ws.release()
+        del ws
+        torch.cuda.empty_cache()
+        ws4 = WeightSet(W, device, replica_tensor_offset(rank, len(W.tensors)), 4)
+        g4q, g4d, _ = ws4.capture()
+        q4 = statistics.median(time_fn(g4q.replay, 5, device))
+        d4 = statistics.median(time_fn(g4d.replay, 5, device))
+        ws4.release()
+        qb4 = n * bytes_per_weight_quant(4)
+        breakdown["ops_4bit"] = {
+            "quantize": {"ms": round(q4, 4), "Gweights_s": round(n / q4 / 1e6, 1),
+                         "GB_s": round(qb4 / q4 / 1e6, 1), "frac_hbm": round(qb4 / q4 / 1e6 / peak, 4)},
+            "dequantize": {"ms": round(d4, 4), "Gweights_s": round(n / d4 / 1e6, 1),
+                           "GB_s": round(qb4 / d4 / 1e6, 1), "frac_hbm": round(qb4 / d4 / 1e6 / peak, 4)}}
+        del ws4
+        torch.cuda.empty_cache()
+        breakdown["gemv_7b_mlp_48_replicas"] = gemv_replica_workload(device, peak)
+        ws = WeightSet(W, device, replica_tensor_offset(rank, len(W.tensors)), BITS)
+        ws.capture()
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(ws, args, device, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, rows, passes, dt, nth = cpu_oracle_sample(args.cpu_seconds)
+        cpu = {"value": round(v, 6), "unit": UNIT, "cores": nth, "kind": "oracle",
+               "sample": f"first {rows} rows (x4096, bf16) of tensor l0.q, {passes} passes of "
+                         f"2-bit quantise + dequantise + batch-1 GEMV, {dt:.1f} s"}
+
+    ws.release()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": "llama7b_bf16 weight set (6,476,005,376 weights, 224 tensors), "
+                                   "2-bit quantize + dequantize(bf16) + batch-1 dequant-GEMV per step",
+                       "bits": BITS, "group_size": 128, "seed": W.seed,
+                       "l2": "inputs (12.95 GB) larger than L2; no flush",
+                       "parallelism": f"replica per GPU x{world}"},
+            "roofline": {"bound": "hbm", "kernel": f"cq_{dom}", "achieved": round(achieved, 1),
+                         "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic},
+            "breakdown": breakdown,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "clocks": clocks,
+            "gpu_launches": ws.launches_per_step() * args.steps,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def load_traffic(kernel: str, n_weights: int):
+    """DRAM bytes per launch-unit from the committed ncu summary, scaled to this launch, or
+    None if the summary is missing or was taken on a different kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        ent = d[kernel]
+        from hadamard_codebook_bit_b200 import build as b
+        if ent.get("source_hash") != b.source_hash():
+            return None
+        return round(ent["dram_bytes_per_weight"] * n_weights)
+    except (OSError, KeyError, ValueError, AttributeError):
+        return None
+
+
+def run_e2e(ws, args, device, world):
+    """Same step through the public API with the inputs in pinned HOST memory: each step
+    copies the bf16 weights and the activations host->device, runs quantise / dequantise /
+    GEMV, and reads packed + norms + dequantised weights + y back to pinned host memory."""
+    import torch
+    steps = max(1, min(args.steps, 3))
+    w_h = torch.empty_like(ws.w, device="cpu").pin_memory()
+    w_h.copy_(ws.w)
+    x_h = {c: x.cpu().pin_memory() for c, x in ws.x.items()}
+    packed_h = torch.empty_like(ws.packed, device="cpu").pin_memory()
+    norms_h = torch.empty_like(ws.norms, device="cpu").pin_memory()
+    out_h = torch.empty_like(ws.out, device="cpu").pin_memory()
+    y_h = torch.empty_like(ws.y, device="cpu").pin_memory()
+    h2d = ws.w.numel() * 2 + sum(x.numel() * 2 for x in ws.x.values())
+    d2h = ws.packed.numel() + ws.norms.numel() * 2 + ws.out.numel() * 2 + ws.y.numel() * 4
+
+    def step():
+        ws.w.copy_(w_h, non_blocking=True)
+        for c, x in ws.x.items():
+            x.copy_(x_h[c], non_blocking=True)
+        for g in ws.graphs:
+            g.replay()
+        packed_h.copy_(ws.packed, non_blocking=True)
+        norms_h.copy_(ws.norms, non_blocking=True)
+        out_h.copy_(ws.out, non_blocking=True)
+        y_h.copy_(ws.y, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize(device)
+    barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize(device)
+    barrier()
+    ms = max_over_ranks(a.elapsed_time(b), device)
+    return {"value": round(world * ws.n * steps / (ms / 1e3) / 1e9, 3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": round(ms / steps, 2)}
+
+
+# ------------------------------------------------------------------------------------------
+# the reference arm: the CPU oracle, as it stands, on a bounded sample
+# ------------------------------------------------------------------------------------------
+
+def run_reference_arm(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    per_step = max(1.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    rows = None
+    nth = oracle.default_threads()
+    passes = 0
+    for i in range(args.warmup + args.steps):
+        v, rows, passes, dt, nth = cpu_oracle_sample(per_step)
+        if i >= args.warmup:
+            vals.append(v)
+    value = statistics.median(vals)
+    sample = (f"first {rows} rows (x4096, bf16) of tensor l0.q per step, {passes} passes of "
+              f"2-bit quantise + dequantise + batch-1 GEMV (~{per_step:.0f} s per step)")
+    from synth import workloads as wlm
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(rows * 4096 * passes / (value * 1e9) * 1e3, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "llama7b_bf16 weight set, bounded sample (see cpu_baseline.sample)",
+                   "bits": BITS, "group_size": 128, "seed": wlm.LLAMA_7B.seed},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": nth, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ncu_case(args):
+    """Small fixed launches for a detailed ncu capture: a 32768x4096 bf16 tensor (256 MiB,
+    larger than L2) quantised and dequantised, then one 11008x4096 2-bit GEMV at batch 1
+    and 8.  Each kernel launches 1 + 3 times (the first is a warm-up)."""
+    import torch
+    import hadamard_codebook_bit_b200 as cq
+    import synth
+    device = torch.device("cuda:0")
+    rows, cols, bits = 32768, 4096, args.ncu_bits
+    w = torch.empty((rows, cols), dtype=torch.bfloat16, device=device)
+    synth.fill_normal_(w, 3, 0, 0.02)
+    packed, norms = cq.empty_packed(rows, cols, bits, device)
+    out = torch.empty_like(w)
+    for _ in range(4):
+        cq.quantize(w, bits, out=(packed, norms))
+    for _ in range(4):
+        cq.dequantize(packed, norms, rows, cols, bits, out=out)
+    g_rows, g_cols = 11008, 4096
+    pk, nm = cq.quantize(w.view(-1)[:g_rows * g_cols].view(g_rows, g_cols), 2)
+    for batch in (1, 8):
+        x = torch.empty((batch, g_cols), dtype=torch.bfloat16, device=device)
+        synth.fill_normal_(x, 4, 100, 1.0)
+        for _ in range(4):
+            cq.dequant_gemv(pk, nm, g_rows, g_cols, 2, x)
+    torch.cuda.synchronize(device)
+    print(json.dumps({"ncu_case": "done", "rows": rows, "cols": cols, "bits": bits}))
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["cq", "reference"], default="cq")
+    ap.add_argument("--quick", action="store_true", help="skip the 4-bit and GEMV-replica extras")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ncu-case", action="store_true",
+                    help="run the small fixed launches used for detailed ncu captures and exit")
+    ap.add_argument("--ncu-bits", type=int, default=2)
+    args = ap.parse_args()
+    if args.ncu_case:
+        run_ncu_case(args)
+        return
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference_arm(args)
+    else:
+        run_cuda_arm(args)
+
+
+if __name__ == "__main__":
+    main()

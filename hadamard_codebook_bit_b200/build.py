@@ -39,6 +39,17 @@ def _deps() -> list[str]:
     return out
 
 
+def source_hash() -> str:
+    """SHA-256 over the kernel sources and the public header (identifies a kernel build)."""
+    import hashlib
+    h = hashlib.sha256()
+    for path in sorted(_deps()):
+        h.update(os.path.basename(path).encode())
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def _compile(src: str, verbose: bool) -> tuple[str, str]:
     path = os.path.join(CSRC, src)
     obj = os.path.join(BUILD, src + ".o")

@@ -70,7 +70,7 @@ def roundtrip_check(ora, w_dev, bits, what, codebook=None, out_dtypes=("f32", "b
         parity.check_dequant_f32(to_np(out), ref, cols, what + " f32")
     if "bf16" in out_dtypes:
         out = cq.dequantize(packed, norms, rows, cols, bits, codebook=cb_dev, out_dtype=torch.bfloat16)
-        parity.check_dequant_bf16(to_np(out), ref, what + " bf16")
+        parity.check_dequant_bf16(to_np(out), ref, cols, what + " bf16")
     return g_packed, g_norms, w64, flips
 
 
@@ -156,7 +156,7 @@ def test_llama7b_sampled(ora, bits):
     pk = torch.from_numpy(g_packed).to(DEV)
     nm = torch.from_numpy(g_norms.view(np.float16)).to(DEV)
     deq = cq.dequantize(pk, nm, rows, 128, bits, out_dtype=torch.bfloat16)
-    parity.check_dequant_bf16(to_np(deq), ora.dequantize(g_packed, g_norms, rows, 128, bits), "llama7b")
+    parity.check_dequant_bf16(to_np(deq), ora.dequantize(g_packed, g_norms, rows, 128, bits), 128, "llama7b")
 
 
 @pytest.mark.parametrize("ti", [0, 1])
@@ -266,4 +266,4 @@ def test_more_than_2g_elements_sampled(ora):
     parity.check_indices(g_packed, o_packed, u, 2, cq.codebook(2), "2G")
     parity.check_norms(g_norms, o_norms, parity.group_norms(parity.bf16_to_f64(w_np), cols))
     ref = ora.dequantize(g_packed, g_norms, len(sel), cols, 2)
-    parity.check_dequant_bf16(to_np(out[torch.from_numpy(sel).to(DEV)]), ref, "2G deq")
+    parity.check_dequant_bf16(to_np(out[torch.from_numpy(sel).to(DEV)]), ref, cols, "2G deq")
