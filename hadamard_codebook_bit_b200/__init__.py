@@ -27,8 +27,9 @@ _STATUS = {0: "CQ_OK", 1: "CQ_ERR_INVALID_ARG", 2: "CQ_ERR_UNSUPPORTED", 3: "CQ_
            4: "CQ_ERR_ALIGNMENT", 5: "CQ_ERR_WORKSPACE"}
 
 # Every symbol include/cq.h declares (checked by the CPU test suite).
-EXPORTS = ("cq_status_string", "cq_version", "cq_codebook", "cq_packed_bytes", "cq_norm_bytes",
-           "cq_quantize", "cq_dequantize", "cq_dequant_gemv", "cq_gemv_workspace_bytes")
+EXPORTS = ("cq_status_string", "cq_version", "cq_device_status", "cq_codebook", "cq_packed_bytes",
+           "cq_norm_bytes", "cq_quantize", "cq_dequantize", "cq_dequant_gemv",
+           "cq_gemv_workspace_bytes")
 
 
 class CQError(RuntimeError):
@@ -52,6 +53,7 @@ def lib() -> ctypes.CDLL:
         L.cq_status_string.argtypes = [i]
         L.cq_status_string.restype = ctypes.c_char_p
         L.cq_version.restype = i
+        L.cq_device_status.argtypes = [i, P]
         L.cq_codebook.argtypes = [i, i, ctypes.c_ulonglong, P, P]
         L.cq_packed_bytes.argtypes = [ll, ll, i, i]
         L.cq_packed_bytes.restype = sz
@@ -69,6 +71,13 @@ def lib() -> ctypes.CDLL:
 def _check(rc: int, what: str) -> None:
     if rc != 0:
         raise CQError(rc, what)
+
+
+def device_status(reset: bool = False) -> int:
+    """Watchdog word of the current device (0 = no kernel wait ever gave up); synchronises."""
+    v = ctypes.c_uint(0)
+    _check(lib().cq_device_status(int(reset), ctypes.byref(v)), "cq_device_status")
+    return int(v.value)
 
 
 def field_bits(bits: int) -> int:

@@ -3,6 +3,7 @@
 // Host side only: argument validation (before any launch), the per-device default
 // codebook, and dispatch to the kernel launchers.  Nothing here computes on the data.
 #include <cstdint>
+#include <cstdlib>
 #include <mutex>
 
 #include "cq_internal.h"
@@ -17,9 +18,13 @@ constexpr int kMaxDevices = 64;
 // 1 = 2-bit, 2 = 3-bit, 3 = 4-bit.  Filled lazily, once per (device, slot).
 __device__ float g_default_codebooks[4][16];
 
+// Watchdog status of the kernels on this device (bit 0: a bounded wait gave up).
+__device__ unsigned g_status;
+
 std::mutex g_mu;
 bool g_default_ready[kMaxDevices][4];
 int g_sm_count[kMaxDevices];
+unsigned* g_status_ptr[kMaxDevices];
 
 int slot_for_bits(int bits) { return bits == CQ_BITS_TERNARY ? 0 : bits - 1; }
 
@@ -84,6 +89,26 @@ int resolve_codebook(int bits, const float* codebook, const float** cb) {
 
 }  // namespace
 
+unsigned* device_status_ptr() {
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (g_status_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+        g_status_ptr[dev] = static_cast<unsigned*>(p);
+    }
+    return g_status_ptr[dev];
+}
+
+bool tcgen05_enabled() {
+    static const bool on = [] {
+        const char* v = std::getenv("CQ_DISABLE_TCGEN05");
+        return v == nullptr || v[0] == '\0' || (v[0] == '0' && v[1] == '\0');
+    }();
+    return on;
+}
+
 int sm_count() {
     const int dev = current_device();
     if (dev < 0 || dev >= kMaxDevices) return 148;
@@ -114,6 +139,20 @@ const char* cq_status_string(int status) {
 }
 
 int cq_version(void) { return 10000; }
+
+int cq_device_status(int reset, unsigned* status_out) {
+    if (status_out == nullptr) return CQ_ERR_INVALID_ARG;
+    unsigned* p = cq::device_status_ptr();
+    if (p == nullptr) return CQ_ERR_CUDA;
+    unsigned v = 0;
+    if (cudaMemcpy(&v, p, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return CQ_ERR_CUDA;
+    if (reset) {
+        const unsigned zero = 0;
+        if (cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return CQ_ERR_CUDA;
+    }
+    *status_out = v;
+    return CQ_OK;
+}
 
 int cq_codebook(int bits, int group_size, unsigned long long seed, float* out_host, int* n_levels) {
     if (out_host == nullptr || seed > 0xffffffffULL) return CQ_ERR_INVALID_ARG;

@@ -117,13 +117,19 @@ __device__ __forceinline__ float quad_sum(float x) {
 // (equal to the nearest level with ties to the lower index, T_k = midpoint * scale)
 // ---------------------------------------------------------------------------------------
 
+// All-ones when a > b, else zero (a single compare-and-set).
+__device__ __forceinline__ uint32_t set_gt(float a, float b) {
+    uint32_t d;
+    asm("set.gt.u32.f32 %0, %1, %2;" : "=r"(d) : "f"(a), "f"(b));
+    return d;
+}
+
 template <int L>
 __device__ __forceinline__ uint32_t nearest_index(float r, const float (&T)[L - 1]) {
-    if constexpr (L <= 4) {
-        uint32_t idx = 0;
-#pragma unroll
-        for (int k = 0; k < L - 1; ++k) idx += (r > T[k]) ? 1u : 0u;
-        return idx;
+    if constexpr (L == 3) {
+        return 0u - (set_gt(r, T[0]) + set_gt(r, T[1]));
+    } else if constexpr (L == 4) {
+        return 0u - (set_gt(r, T[0]) + set_gt(r, T[1]) + set_gt(r, T[2]));
     } else if constexpr (L == 8) {
         const bool b2 = r > T[3];
         const bool b1 = r > (b2 ? T[5] : T[1]);

@@ -28,6 +28,20 @@ struct Shape {
 };
 
 // Kernel launchers (one per file).  All return cudaSuccess or the launch error.
+// Device-wide status word of the current device (bit 0: a bounded wait inside a kernel gave
+// up).  Returns nullptr if the symbol address cannot be obtained.
+unsigned* device_status_ptr();
+
+// True when the tensor-core (tcgen05 + TMA) implementations are enabled for this process
+// (environment variable CQ_DISABLE_TCGEN05 unset or "0").
+bool tcgen05_enabled();
+
+// Tensor-core quantiser (cq_quantize_tc.cu): bf16 input, cols % 8 == 0.
+bool quantize_tc_supported(int w_dtype, const Shape& s);
+cudaError_t launch_quantize_tc(const void* w, const Shape& s, int bits, const float* codebook,
+                               uint8_t* packed, uint16_t* norms, unsigned* status,
+                               cudaStream_t stream);
+
 cudaError_t launch_quantize(const void* w, int w_dtype, const Shape& s, int bits,
                             const float* codebook, uint8_t* packed, uint16_t* norms,
                             cudaStream_t stream);

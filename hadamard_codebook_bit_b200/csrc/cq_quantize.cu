@@ -182,6 +182,11 @@ cudaError_t launch_dtype(int w_dtype, int mode, const void* w, const Shape& sh, 
 cudaError_t launch_quantize(const void* w, int w_dtype, const Shape& sh, int bits,
                             const float* codebook, uint8_t* packed, uint16_t* norms,
                             cudaStream_t stream) {
+    if (tcgen05_enabled() && quantize_tc_supported(w_dtype, sh)) {
+        unsigned* status = device_status_ptr();
+        if (status != nullptr)
+            return launch_quantize_tc(w, sh, bits, codebook, packed, norms, status, stream);
+    }
     const int chunk = (w_dtype == CQ_BF16) ? 8 : 4;  // elements per 16 bytes
     const int mode = (sh.cols % 128 == 0) ? kFlat : (sh.cols % chunk == 0) ? kVector : kScalar;
     switch (bits) {

@@ -1,0 +1,315 @@
+// cq_quantize_tc.cu -- bf16 W -> packed indices + fp16 norms with the rotation on the
+// fifth-generation tensor cores (tcgen05), for bf16 inputs whose rows start on 16 bytes.
+//
+// Same arithmetic as cq_quantize.cu (page "Cactus Quants CQ2-bit Quantization", "The CQ2-bit
+// Implementation Pipeline" steps 1-4): the rotation r = H_int v of 128 groups at a time is
+// the product  R[128 groups x 128] = V[128 x 128] . H_int[128 x 128]  (H symmetric), a bf16 x
+// bf16 MMA with exact +-1 weights and fp32 accumulation, which is how the pages write the
+// rotation ("rot @ H", page "How CQ2-bit Quantization Contributes to Needle 2's Small
+// Footprint", "Hadamard Rotation").
+//
+// Persistent kernel, one 320-thread CTA per SM:
+//   warp 0      TMA producer: 128 x 128 bf16 tiles (two 64-column boxes, 128-byte swizzle)
+//               into a 4-stage shared-memory ring;
+//   warp 1      owns 256 TMEM columns; one lane issues 8 tcgen05.mma (M=128, N=128, K=16)
+//               per tile into one of two TMEM accumulators, then commits to the stage's
+//               "empty" barrier and the accumulator's "full" barrier;
+//   warps 2-9   two epilogue groups of four warps (one per TMEM lane quadrant) take
+//               alternating tiles: each thread reads its group's 128 rotated values from
+//               TMEM, forms the norm, the thresholds m_k * ||r||, the indices, and stores
+//               the packed block and the fp16 norm.
+// H_int lives in shared memory in the same swizzled K-major layout (built once per CTA).
+//
+// Tile -> groups: the tensor map views W as [R_eff rows x C_eff cols]; tile (rb, j) covers
+// rows 128 rb .. 128 rb + 127 and columns 128 j .. 128 j + 127 (zero filled past the edges,
+// which is the pages' zero padding); its lane m is group (128 rb + m) * G_eff + j.  With
+// cols % 128 == 0 the whole matrix is viewed as [groups x 128] (G_eff = 1), so one tile is
+// 128 consecutive groups and the packed output of a tile is one contiguous block.
+#include <algorithm>
+#include <mutex>
+
+#include "cq_device.cuh"
+#include "cq_internal.h"
+#include "cq_sm100.cuh"
+
+namespace cq {
+namespace {
+
+using namespace dev;
+using namespace sm100;
+
+constexpr int kEpiGroups = 4;                          // epilogue warpgroups = TMEM accumulators
+constexpr int kTcThreads = 64 + 128 * kEpiGroups;      // producer + MMA warps, then epilogue
+constexpr int kTile = 128;                 // groups per tile (MMA M) = elements per group (K, N)
+constexpr int kStagesTc = 4;
+constexpr int kTileBytes = kTile * kTile * 2;  // 32 KiB of bf16
+constexpr int kHalfBytes = kTileBytes / 2;     // one 64-column box
+constexpr int kTmemCols = 128 * kEpiGroups;    // one fp32 accumulator of 128 columns per group
+constexpr uint32_t kIdesc = idesc_bf16_f32(kTile, kTile);
+
+struct TcShape {
+    long long r_eff, g_eff, tiles_r, tiles;
+};
+
+// Byte offset of element (row, k) of a 128 x 128 bf16 K-major tile stored as two 64-column
+// halves, each with the 128-byte swizzle (16-byte chunk index XOR row % 8).
+__device__ __forceinline__ int sw128_offset(int row, int k) {
+    const int half = k >> 6, kl = k & 63;
+    return half * kHalfBytes + row * 128 + (((kl >> 3) ^ (row & 7)) << 4) + (kl & 7) * 2;
+}
+
+template <int B, int L>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    quantize_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcShape sh,
+                       const float* __restrict__ codebook, uint8_t* __restrict__ packed,
+                       uint16_t* __restrict__ norms, unsigned* __restrict__ status) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full_bar[kStagesTc], empty_bar[kStagesTc];
+    __shared__ __align__(8) uint64_t tfull_bar[kEpiGroups], tempty_bar[kEpiGroups];
+    __shared__ uint32_t tmem_slot;
+
+    // 1024-byte aligned region: H_int, then the stage ring
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* hmat = smem;
+    uint8_t* ring = smem + kTileBytes;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // H_int (+1 = 0x3F80, -1 = 0xBF80 in bf16), row n = output element, column k = input element
+    for (int item = threadIdx.x; item < kTile * 16; item += kTcThreads) {
+        const int n = item >> 4, c16 = item & 15;  // 16 chunks of 8 elements per row
+        uint32_t w4[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const int k0 = c16 * 8 + 2 * p;
+            const uint32_t lo = (__popc(n & k0) & 1) ? 0xBF80u : 0x3F80u;
+            const uint32_t hi = (__popc(n & (k0 + 1)) & 1) ? 0xBF80u : 0x3F80u;
+            w4[p] = lo | (hi << 16);
+        }
+        *reinterpret_cast<uint4*>(hmat + sw128_offset(n, c16 * 8)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
+    fence_proxy_async_smem();
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStagesTc; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int a = 0; a < kEpiGroups; ++a) {
+            mbar_init(&tfull_bar[a], 1);
+            mbar_init(&tempty_bar[a], 4);
+        }
+        fence_mbar_init();
+        prefetch_tensormap(&tmap);
+    }
+    if (warp == 1) tmem_alloc(&tmem_slot, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = tmem_slot;
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            int i = 0;
+            for (long long t = blockIdx.x; t < sh.tiles; t += gridDim.x, ++i) {
+                const int st = i % kStagesTc;
+                const uint32_t ph = (i / kStagesTc) & 1;
+                if (!mbar_wait(&empty_bar[st], ph ^ 1, status)) break;
+                const int rb = static_cast<int>(t % sh.tiles_r);
+                const int j = static_cast<int>(t / sh.tiles_r);
+                uint8_t* dst = ring + st * kTileBytes;
+                mbar_arrive_expect_tx(&full_bar[st], kTileBytes);
+                tma_load_2d(dst, &tmap, kTile * j, kTile * rb, &full_bar[st]);
+                tma_load_2d(dst + kHalfBytes, &tmap, kTile * j + 64, kTile * rb, &full_bar[st]);
+            }
+            // drain: wait (bounded) until every stage this CTA filled has been consumed
+            for (int k = 0; k < kStagesTc && k < i; ++k) {
+                const int ii = i - 1 - k;
+                mbar_wait(&empty_bar[ii % kStagesTc], (ii / kStagesTc) & 1, status);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            int i = 0;
+            for (long long t = blockIdx.x; t < sh.tiles; t += gridDim.x, ++i) {
+                const int st = i % kStagesTc;
+                const int acc = i % kEpiGroups;
+                if (!mbar_wait(&full_bar[st], (i / kStagesTc) & 1, status)) break;
+                if (!mbar_wait(&tempty_bar[acc], ((i / kEpiGroups) & 1) ^ 1, status)) break;
+                tc_fence_after();
+                const uint32_t a_base = smem_u32(ring + st * kTileBytes);
+                const uint32_t b_base = smem_u32(hmat);
+#pragma unroll
+                for (int k = 0; k < kTile / 16; ++k) {
+                    const uint32_t off = (k >> 2) * kHalfBytes + (k & 3) * 32;
+                    mma_f16(tbase + acc * kTile, smem_desc_sw128(a_base + off),
+                            smem_desc_sw128(b_base + off), kIdesc, k > 0);
+                }
+                mma_commit(&empty_bar[st]);
+                mma_commit(&tfull_bar[acc]);
+            }
+        }
+    } else {
+        // ---------------- epilogue ----------------
+        const int e = (warp - 2) >> 2;   // accumulator this group serves (tiles i = e mod 4)
+        const int quad = warp & 3;       // TMEM lanes 32 quad .. 32 quad + 31
+        const int m = quad * 32 + lane;  // group within the tile
+        float mid[L - 1];
+#pragma unroll
+        for (int k = 0; k < L - 1; ++k) mid[k] = 0.5f * (__ldg(codebook + k) + __ldg(codebook + k + 1));
+        int i = e;
+        for (long long t = blockIdx.x + static_cast<long long>(e) * gridDim.x; t < sh.tiles;
+             t += static_cast<long long>(kEpiGroups) * gridDim.x, i += kEpiGroups) {
+            // warp-uniform decision: the TMEM loads below are .sync.aligned
+            const bool ok = __all_sync(kFullMask, mbar_wait(&tfull_bar[e], (i / kEpiGroups) & 1, status));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t taddr = tbase + (static_cast<uint32_t>(quad * 32) << 16) + e * kTile;
+            const long long rb = t % sh.tiles_r, j = t / sh.tiles_r;
+            const long long row = rb * kTile + m;
+            const long long gid = row * sh.g_eff + j;
+            // pass 1: the squared norm of the rotated group (32 TMEM columns at a time,
+            // four independent partial sums)
+            float ps[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+            for (int c = 0; c < kTile / 32; ++c) {
+                float v[32];
+                tmem_ld32(taddr + 32 * c, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int q = 0; q < 32; ++q) ps[q & 3] = fmaf(v[q], v[q], ps[q & 3]);
+            }
+            const float ss = (ps[0] + ps[1]) + (ps[2] + ps[3]);
+            const float nrm = sqrtf(ss);
+            float T[L - 1];
+#pragma unroll
+            for (int k = 0; k < L - 1; ++k) T[k] = nrm > 0.0f ? mid[k] * nrm : mid[k];
+            // pass 2: indices, B words per 32 elements
+            uint32_t words[4 * B];
+#pragma unroll
+            for (int c = 0; c < kTile / 32; ++c) {
+                float v[32];
+                tmem_ld32(taddr + 32 * c, v);
+                tmem_ld_wait();
+                if constexpr (B == 3) {
+#pragma unroll
+                    for (int w = 0; w < B; ++w) words[B * c + w] = 0u;
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) {
+                        const uint32_t idx = nearest_index<L>(v[q], T);
+                        const int bit = B * q, w = B * c + (bit >> 5), sh2 = bit & 31;
+                        words[w] |= idx << sh2;
+                        if (sh2 + B > 32) words[w + 1] |= idx >> (32 - sh2);
+                    }
+                } else {
+                    // 32 / B fields per word, accumulated top-down: word = (word << B) + idx
+#pragma unroll
+                    for (int w = 0; w < B; ++w) {
+                        uint32_t acc = 0u;
+#pragma unroll
+                        for (int q = 32 / B - 1; q >= 0; --q)
+                            acc = (acc << B) + nearest_index<L>(v[w * (32 / B) + q], T);
+                        words[B * c + w] = acc;
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty_bar[e]);
+            if (row >= sh.r_eff) continue;
+            uint4* dst = reinterpret_cast<uint4*>(packed + gid * (16 * B));
+#pragma unroll
+            for (int p = 0; p < B; ++p)
+                dst[p] = make_uint4(words[4 * p], words[4 * p + 1], words[4 * p + 2], words[4 * p + 3]);
+            norms[gid] = __half_as_ushort(__float2half_rn(sqrtf(ss * 0.0078125f)));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tbase, kTmemCols);
+    }
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                              CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                              CUtensorMapFloatOOBfill);
+
+EncodeFn encode_fn() {
+    static EncodeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeFn>(p);
+    });
+    return fn;
+}
+
+template <int B, int L>
+cudaError_t launch_tc(const CUtensorMap& map, const TcShape& ts, const float* cb, uint8_t* packed,
+                      uint16_t* norms, unsigned* status, cudaStream_t st) {
+    const int smem = (1 + kStagesTc) * kTileBytes + 1024;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    static unsigned long long configured = 0;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(configured & bit)) {
+        e = cudaFuncSetAttribute(quantize_tc_kernel<B, L>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        configured |= bit;
+    }
+    const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(ts.tiles, sm_count())));
+    quantize_tc_kernel<B, L><<<grid, kTcThreads, smem, st>>>(map, ts, cb, packed, norms, status);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool quantize_tc_supported(int w_dtype, const Shape& sh) {
+    if (w_dtype != CQ_BF16 || sh.cols % 8 != 0) return false;
+    const bool flat = sh.cols % kTile == 0;
+    const long long r_eff = flat ? sh.total_groups : sh.rows;
+    if (r_eff >= (1LL << 31)) return false;
+    return encode_fn() != nullptr;
+}
+
+cudaError_t launch_quantize_tc(const void* w, const Shape& sh, int bits, const float* codebook,
+                               uint8_t* packed, uint16_t* norms, unsigned* status,
+                               cudaStream_t stream) {
+    const bool flat = sh.cols % kTile == 0;
+    TcShape ts;
+    ts.r_eff = flat ? sh.total_groups : sh.rows;
+    const long long c_eff = flat ? kTile : sh.cols;
+    ts.g_eff = flat ? 1 : sh.groups_per_row;
+    ts.tiles_r = (ts.r_eff + kTile - 1) / kTile;
+    ts.tiles = ts.tiles_r * ts.g_eff;
+
+    CUtensorMap map;
+    const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(c_eff), static_cast<cuuint64_t>(ts.r_eff)};
+    const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(c_eff) * 2};
+    const cuuint32_t box[2] = {64, kTile};
+    const cuuint32_t estride[2] = {1, 1};
+    const CUresult r = encode_fn()(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(w), gdim,
+                                   gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    switch (bits) {
+        case CQ_BITS_TERNARY: return launch_tc<2, 3>(map, ts, codebook, packed, norms, status, stream);
+        case 2: return launch_tc<2, 4>(map, ts, codebook, packed, norms, status, stream);
+        case 3: return launch_tc<3, 8>(map, ts, codebook, packed, norms, status, stream);
+        default: return launch_tc<4, 16>(map, ts, codebook, packed, norms, status, stream);
+    }
+}
+
+}  // namespace cq

@@ -75,6 +75,18 @@ const char* cq_status_string(int status);
 int cq_version(void);
 
 /*
+ * cq_device_status -- watchdog word of the current device.
+ *
+ * The tensor-core kernels coordinate their warps through shared-memory barriers; every wait
+ * on one gives up after a few seconds instead of spinning forever, sets bit 0 of this word,
+ * and the kernel returns early (its outputs are then incomplete).  This call copies the
+ * word to *status_out (0 = no wait ever gave up) and clears it when `reset` is nonzero.
+ * It synchronises with the device (a blocking copy), so it is a diagnostic, not for hot
+ * paths.  Returns CQ_OK, CQ_ERR_INVALID_ARG (status_out NULL) or CQ_ERR_CUDA.
+ */
+int cq_device_status(int reset, unsigned* status_out);
+
+/*
  * cq_codebook -- the default codebook for `bits` (host routine, setup only).
  *
  * Page "How Quantization Codebooks Are Trained in Cactus Quants": Lloyd-Max (1-D k-means)
@@ -159,6 +171,12 @@ int cq_dequantize(const unsigned char* packed, const unsigned short* norms, long
  * fp32.  The memory-bandwidth motive is page "Performance Differences Between 2-Bit and
  * 4-Bit Quantization in Needle", "Model Size and Memory Bandwidth".
  *
+ * Arithmetic: the products run on the tensor cores in fp16 with fp32 accumulation.  The
+ * codewords are scaled by one exact power of two per call and each rotated activation
+ * group by its own power of two (largest magnitude in [2^13, 2^14)) before rounding to
+ * fp16, so any finite input is in range; the relative error of y is about 2e-4 (bound
+ * 1e-3 per output vector).  Summation order is fixed: repeated calls give identical bits.
+ *
  *   packed, norms  DEVICE, W quantised as [rows, cols] (rows = outputs, cols = inputs)
  *   rows, cols     >= 0
  *   bits           CQ_BITS_TERNARY, 2, 3 or 4
@@ -167,9 +185,10 @@ int cq_dequantize(const unsigned char* packed, const unsigned short* norms, long
  *   x              DEVICE bf16 [batch, cols], row-major
  *   batch          1..8
  *   y              DEVICE fp32 [batch, rows], row-major, overwritten
- *   workspace      DEVICE scratch of at least cq_gemv_workspace_bytes(cols, batch) bytes,
- *                  16-byte aligned; its contents on entry are ignored and on return are
- *                  unspecified.  Calls that overlap in time must not share a workspace.
+ *   workspace      DEVICE scratch of at least cq_gemv_workspace_bytes(cols, batch) bytes
+ *                  (2080 bytes per 128 columns), 16-byte aligned; its contents on entry are
+ *                  ignored and on return are unspecified.  Calls that overlap in time must
+ *                  not share a workspace.
  */
 int cq_dequant_gemv(const unsigned char* packed, const unsigned short* norms, long long rows,
                     long long cols, int bits, int group_size, const float* codebook,

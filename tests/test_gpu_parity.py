@@ -267,3 +267,8 @@ def test_more_than_2g_elements_sampled(ora):
     parity.check_norms(g_norms, o_norms, parity.group_norms(parity.bf16_to_f64(w_np), cols))
     ref = ora.dequantize(g_packed, g_norms, len(sel), cols, 2)
     parity.check_dequant_bf16(to_np(out[torch.from_numpy(sel).to(DEV)]), ref, cols, "2G deq")
+
+
+def test_zz_no_kernel_wait_gave_up():
+    """Every bounded wait inside the tensor-core kernels completed during this module."""
+    assert cq.device_status() == 0
