@@ -186,7 +186,7 @@ int cq_dequantize(const unsigned char* packed, const unsigned short* norms, long
  *   batch          1..8
  *   y              DEVICE fp32 [batch, rows], row-major, overwritten
  *   workspace      DEVICE scratch of at least cq_gemv_workspace_bytes(cols, batch) bytes
- *                  (2080 bytes per 128 columns), 16-byte aligned; its contents on entry are
+ *                  (2080 bytes per 128 columns plus 48), 16-byte aligned; its contents on entry are
  *                  ignored and on return are unspecified.  Calls that overlap in time must
  *                  not share a workspace.
  */

@@ -82,8 +82,8 @@ def test_byte_counts_match_oracle(oracle_lib, rows, cols, bits, L):
 def test_byte_counts_edge_cases(L):
     assert cq.packed_bytes(0, 5, 2) == 0 and cq.norm_bytes(5, 0) == 0
     assert cq.packed_bytes(-1, 5, 2) == 0 and cq.packed_bytes(5, 5, 7) == 0
-    def ws(G):
-        return -(-(G * 2080) // 256) * 256
+    def ws(G):  # B-operand fragments, per-column exponents, one 48-byte codeword table
+        return -(-(G * 2080 + 48) // 256) * 256
     assert cq.gemv_workspace_bytes(4096, 1) == ws(32) == cq.gemv_workspace_bytes(4096, 8)
     assert cq.gemv_workspace_bytes(11008, 8) == ws(86)
     assert cq.gemv_workspace_bytes(1, 3) == ws(1)
