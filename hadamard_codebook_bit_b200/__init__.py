@@ -29,7 +29,7 @@ _STATUS = {0: "CQ_OK", 1: "CQ_ERR_INVALID_ARG", 2: "CQ_ERR_UNSUPPORTED", 3: "CQ_
 # Every symbol include/cq.h declares (checked by the CPU test suite).
 EXPORTS = ("cq_status_string", "cq_version", "cq_device_status", "cq_codebook", "cq_packed_bytes",
            "cq_norm_bytes", "cq_quantize", "cq_dequantize", "cq_dequant_gemv",
-           "cq_gemv_workspace_bytes")
+           "cq_gemv_workspace_bytes", "cq_dequant_gemv_static")
 
 
 class CQError(RuntimeError):
@@ -64,6 +64,7 @@ def lib() -> ctypes.CDLL:
         L.cq_dequant_gemv.argtypes = [P, P, ll, ll, i, i, P, P, i, P, P, sz, P]
         L.cq_gemv_workspace_bytes.argtypes = [ll, i]
         L.cq_gemv_workspace_bytes.restype = sz
+        L.cq_dequant_gemv_static.argtypes = [P, P, ll, ll, i, i, P, P, i, P, P]
         _lib = L
     return _lib
 
@@ -214,4 +215,27 @@ def dequant_gemv(packed, norms, rows: int, cols: int, bits: int, x, group_size: 
                                      _dev_ptr(workspace, "workspace"),
                                      workspace.numel() * workspace.element_size(),
                                      _stream(packed.device)), "cq_dequant_gemv")
+    return y
+
+
+def dequant_gemv_static(packed, norms, rows: int, cols: int, bits: int, x,
+                        group_size: int = GROUP_SIZE, codebook=None, y=None):
+    """cq_dequant_gemv_static: the GEMV with the library's built-in scratch (cols <= 32768),
+    for callers that must not allocate device memory."""
+    torch = _torch()
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    if x.dtype != torch.bfloat16:
+        raise ValueError("x must be bfloat16")
+    if norms.dtype != torch.float16:
+        raise ValueError("norms must be float16")
+    batch = x.shape[0]
+    if y is None:
+        y = torch.empty((batch, rows), dtype=torch.float32, device=packed.device)
+    with torch.cuda.device(packed.device):
+        _check(lib().cq_dequant_gemv_static(_dev_ptr(packed, "packed"), _dev_ptr(norms, "norms"),
+                                            rows, cols, bits, group_size,
+                                            _cb_ptr(codebook, packed.device), _dev_ptr(x, "x"),
+                                            batch, _dev_ptr(y, "y"), _stream(packed.device)),
+               "cq_dequant_gemv_static")
     return y

@@ -22,7 +22,7 @@ BUILD = os.path.join(ROOT, "_build", "libcq")
 LIB = os.path.join(PKG, "libcq.so")
 
 SOURCES = ["cq_api.cu", "cq_quantize.cu", "cq_quantize_tc.cu", "cq_dequantize.cu", "cq_gemv.cu",
-           "cq_codebook.cpp"]
+           "cq_gemv_static.cu", "cq_codebook.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -198,6 +198,30 @@ int cq_dequant_gemv(const unsigned char* packed, const unsigned short* norms, lo
 /* Workspace bytes cq_dequant_gemv needs for this cols and batch (0 if invalid or cols == 0). */
 size_t cq_gemv_workspace_bytes(long long cols, int batch);
 
+/*
+ * cq_dequant_gemv_static -- cq_dequant_gemv without a workspace argument.
+ *
+ * No counterpart on the pages: this is a convenience of this library.  Some callers cannot
+ * allocate device memory at the point where they need the product: code running while a
+ * stream is being captured into a CUDA graph (cudaMalloc is not allowed then), plug-ins
+ * that live inside a host framework and may not bypass its allocator, and C callers with
+ * no device allocator of their own.  This entry point takes its scratch from a fixed array
+ * in the library's own device memory (static, 532,736 bytes, held by every GPU that loads
+ * the library until the process exits) and calls no cudaMalloc, cudaFree or allocating
+ * routine.  Same arguments, semantics and results as cq_dequant_gemv, minus the workspace.
+ *
+ *   cols       at most 32768; larger returns CQ_ERR_WORKSPACE and launches nothing
+ *   set-up     the first call on each device looks up the array's device address (a
+ *              synchronous runtime call); make that first call before any stream capture
+ *   sharing    every call on a device uses the same array, which keeps the last call's
+ *              contents (nothing needs clearing: each call rewrites all it reads); calls
+ *              whose executions overlap on the GPU, e.g. on two unordered streams, race.
+ */
+int cq_dequant_gemv_static(const unsigned char* packed, const unsigned short* norms,
+                           long long rows, long long cols, int bits, int group_size,
+                           const float* codebook, const void* x, int batch, float* y,
+                           void* stream);
+
 #ifdef __cplusplus
 }
 #endif
