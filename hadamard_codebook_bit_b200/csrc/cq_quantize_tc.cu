@@ -58,6 +58,57 @@ __device__ __forceinline__ int sw128_offset(int row, int k) {
     return half * kHalfBytes + row * 128 + (((kl >> 3) ^ (row & 7)) << 4) + (kl & 7) * 2;
 }
 
+// --- 2-bit / ternary packing by sign bits -------------------------------------------------
+// With sorted thresholds T_0 < T_1 (< T_2), s_k = [r > T_k] is the sign bit of e_k = T_k - r
+// (rounding never flips a sign; r == T_k gives +0, i.e. "not greater", the tie going low),
+// and the index sum_k s_k has bits  b1 = s_1,  b0 = s_0 ^ s_1 (^ s_2).  The subtractions run
+// two elements at a time on the FMA pipe (f32x2); the bits are appended into the packed word
+// with funnel shifts, top element first, so element i lands at bits 2i, 2i+1.
+
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t p, uint32_t& lo, uint32_t& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(p));
+}
+__device__ __forceinline__ uint64_t f2sub(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// v[OFF .. OFF+15] -> one word of 16 two-bit codes; pairs (2i, 2i+1) share one f32x2
+// subtraction.
+template <int L, int OFF>
+__device__ __forceinline__ uint32_t pack2_signbits(const float (&v)[32], const float (&T)[L - 1]) {
+    static_assert(L == 3 || L == 4, "2-bit fields");
+    uint64_t tp[L - 1];
+#pragma unroll
+    for (int k = 0; k < L - 1; ++k) tp[k] = f2pack(T[k], T[k]);
+    uint32_t w = 0u;
+#pragma unroll
+    for (int i = 7; i >= 0; --i) {
+        const uint64_t r = f2pack(v[OFF + 2 * i], v[OFF + 2 * i + 1]);
+        uint32_t e0x, e0y, e1x, e1y;
+        f2unpack(f2sub(tp[0], r), e0x, e0y);
+        f2unpack(f2sub(tp[1], r), e1x, e1y);
+        uint32_t lx = e0x ^ e1x, ly = e0y ^ e1y;
+        if constexpr (L == 4) {
+            uint32_t e2x, e2y;
+            f2unpack(f2sub(tp[2], r), e2x, e2y);
+            lx ^= e2x;
+            ly ^= e2y;
+        }
+        w = __funnelshift_l(e1y, w, 1);  // element 2i+1: b1, b0
+        w = __funnelshift_l(ly, w, 1);
+        w = __funnelshift_l(e1x, w, 1);  // element 2i: b1, b0
+        w = __funnelshift_l(lx, w, 1);
+    }
+    return w;
+}
+
 template <int B, int L>
 __global__ void __launch_bounds__(kTcThreads, 1)
     quantize_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcShape sh,
@@ -193,7 +244,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 float v[32];
                 tmem_ld32(taddr + 32 * c, v);
                 tmem_ld_wait();
-                if constexpr (B == 3) {
+                if constexpr (B == 2) {
+                    // ternary = the 2-bit form with a third threshold that nothing exceeds
+                    float T3[3];
+#pragma unroll
+                    for (int k = 0; k < 3; ++k) T3[k] = k < L - 1 ? T[k < L - 1 ? k : 0] : __int_as_float(0x7f800000);
+                    words[2 * c] = pack2_signbits<4, 0>(v, T3);
+                    words[2 * c + 1] = pack2_signbits<4, 16>(v, T3);
+                } else if constexpr (B == 3) {
 #pragma unroll
                     for (int w = 0; w < B; ++w) words[B * c + w] = 0u;
 #pragma unroll
