@@ -21,7 +21,8 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build", "libcq")
 LIB = os.path.join(PKG, "libcq.so")
 
-SOURCES = ["cq_api.cu", "cq_quantize.cu", "cq_quantize_tc.cu", "cq_dequantize.cu", "cq_gemv.cu",
+SOURCES = ["cq_api.cu", "cq_quantize.cu", "cq_quantize_tc.cu", "cq_dequantize.cu",
+           "cq_dequantize_tc.cu", "cq_gemv.cu",
            "cq_gemv_static.cu", "cq_codebook.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -101,6 +101,19 @@ unsigned* device_status_ptr() {
     return g_status_ptr[dev];
 }
 
+EncodeTiledFn tensor_map_encoder() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
 bool tcgen05_enabled() {
     static const bool on = [] {
         const char* v = std::getenv("CQ_DISABLE_TCGEN05");

@@ -170,6 +170,11 @@ cudaError_t launch_dtype(int out_dtype, int mode, const uint8_t* packed, const u
 cudaError_t launch_dequantize(const uint8_t* packed, const uint16_t* norms, const Shape& sh,
                               int bits, const float* codebook, void* out, int out_dtype,
                               cudaStream_t stream) {
+    if (tcgen05_enabled() && dequantize_tc_supported(out_dtype, sh)) {
+        unsigned* status = device_status_ptr();
+        if (status != nullptr)
+            return launch_dequantize_tc(packed, norms, sh, bits, codebook, out, out_dtype, status, stream);
+    }
     const int chunk = (out_dtype == CQ_BF16) ? 8 : 4;
     const int mode = (sh.cols % 128 == 0) ? kFlat : (sh.cols % chunk == 0) ? kVector : kScalar;
     switch (bits) {

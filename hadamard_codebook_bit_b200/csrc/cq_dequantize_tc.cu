@@ -1,0 +1,460 @@
+// cq_dequantize_tc.cu -- packed indices + fp16 norms -> W_hat with the inverse rotation on
+// the fifth-generation tensor cores (tcgen05).
+//
+// Same arithmetic as cq_dequantize.cu (page "Cactus Quants CQ2-bit Quantization", "The CQ2-bit
+// Implementation Pipeline" steps 5-6): w_hat = (n / sqrt(128)) H_int c[idx].  For 128 groups
+// at a time the rotation is the product  D[128 groups x 128] = C[128 x 128] . H_int  (H
+// symmetric), where C holds the codewords.  Each codeword, scaled by an exact power of two
+// 2^cs, is split into two fp16 values hi + lo that sum to it within 2^-22 relative, so two
+// fp16 MMAs with exact +-1 weights and fp32 accumulation give the fp32 result.
+//
+// Persistent kernel, one 320-thread CTA per SM (all 512 TMEM columns):
+//   warp 0      bulk-copies each tile's packed blocks (128 groups, contiguous) into a
+//               4-stage shared-memory ring;
+//   warp 1      owns TMEM; one lane issues per tile 16 tcgen05.mma (M=128, N=128, K=16):
+//               8 for the hi plane, 8 for the lo plane, A read from TMEM, B = H_int from
+//               shared memory, into the tile slot's fp32 accumulator;
+//   warps 2-9   two decode/epilogue warpgroups, one TMEM slot each (A hi 64 columns, A lo 64,
+//               D 128), taking alternating tiles: a thread decodes its group's codes into
+//               fp16 pairs with byte permutes, writes them to TMEM (tcgen05.st), and after the
+//               MMAs reads its group's 128 results back, scales them by the norm and stores.
+//
+// K order of a 2-bit group.  The MMA contracts over the 128 input elements in any order as
+// long as A and B agree: column k = 16 w + 4 p + q of A holds element e = 16 w + 4 q + p, the
+// code at bit 2p of byte q of packed word w, so four consecutive columns come from one
+// shift + mask, and row n of the shared-memory B holds H_int[n][e(k)].
+#include <algorithm>
+#include <cstring>
+
+#include "cq_device.cuh"
+#include "cq_internal.h"
+#include "cq_sm100.cuh"
+
+namespace cq {
+namespace {
+
+using namespace dev;
+using namespace sm100;
+
+constexpr int kDqThreads = 64 + 256;
+constexpr int kTile = 128;
+constexpr int kStagesDq = 4;
+constexpr int kSlotCols = 256;                  // A hi (64) + A lo (64) + D (128)
+constexpr int kTmemColsDq = 2 * kSlotCols;
+constexpr int kHBytes = kTile * kTile * 2;      // fp16 H_int, two 64-column swizzled halves
+constexpr int kHHalf = kHBytes / 2;
+constexpr uint32_t kIdescDq = idesc_f16_f32(kTile, kTile);
+
+struct DqShape {
+    long long total;   // groups
+    long long cols;    // columns of W
+    long long G;       // groups per row
+    long long tiles;   // ceil(total / 128)
+    int flat;          // cols % 128 == 0: group g's output starts at element 128 g
+};
+
+// Element of the group held by MMA column k.
+template <int B>
+__device__ __forceinline__ int elem_of_col(int k) {
+    if constexpr (B == 2) {
+        const int w = k >> 4, p = (k >> 2) & 3, q = k & 3;
+        return 16 * w + 4 * q + p;
+    } else {
+        return k;
+    }
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+__device__ __forceinline__ uint32_t mad_hi(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+template <bool kBF16>
+__device__ __forceinline__ void store_chunk(void* out, long long elem, const float (&v)[32], int off,
+                                            float scale) {
+    // 8 (bf16) or 4 (fp32) consecutive values = 16 bytes
+    if constexpr (kBF16) {
+        uint4 o;
+        o.x = pack_bf16x2(v[off + 0] * scale, v[off + 1] * scale);
+        o.y = pack_bf16x2(v[off + 2] * scale, v[off + 3] * scale);
+        o.z = pack_bf16x2(v[off + 4] * scale, v[off + 5] * scale);
+        o.w = pack_bf16x2(v[off + 6] * scale, v[off + 7] * scale);
+        st_stream16(static_cast<uint16_t*>(out) + elem, o);
+    } else {
+        uint4 o;
+        o.x = __float_as_uint(v[off + 0] * scale);
+        o.y = __float_as_uint(v[off + 1] * scale);
+        o.z = __float_as_uint(v[off + 2] * scale);
+        o.w = __float_as_uint(v[off + 3] * scale);
+        st_stream16(static_cast<float*>(out) + elem, o);
+    }
+}
+
+// Output staging for the tensor-map store: per decode group one [128 rows x 128] tile of the
+// output type, as 128-byte-wide boxes of 128 rows with the 128-byte swizzle (conflict-free
+// per-row writes; the TMA unit undoes the swizzle on the way out).
+template <bool kBF16>
+struct OutTile {
+    static constexpr int kBoxes = kBF16 ? 2 : 4;        // 64 bf16 or 32 fp32 per 128-byte box
+    static constexpr int kPerBox = kBF16 ? 64 : 32;
+    static constexpr int kBoxBytes = kTile * 128;
+    static constexpr int kBytes = kBoxes * kBoxBytes;
+    // byte offset of 16-byte chunk `chunk` (of 8 bf16 / 4 fp32 values) of row m
+    __device__ static int chunk_offset(int m, int chunk) {
+        constexpr int kChunksPerBox = 8;
+        const int box = chunk / kChunksPerBox, c = chunk % kChunksPerBox;
+        return box * kBoxBytes + m * 128 + ((c ^ (m & 7)) << 4);
+    }
+};
+
+template <int B, int L, bool kBF16>
+__global__ void __launch_bounds__(kDqThreads, 1)
+    dequantize_tc_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ norms,
+                         DqShape sh, const float* __restrict__ codebook, void* __restrict__ out,
+                         unsigned* __restrict__ status, const __grid_constant__ CUtensorMap omap) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full_bar[kStagesDq], empty_bar[kStagesDq];
+    __shared__ __align__(8) uint64_t afull_bar[2], dfull_bar[2];
+    __shared__ uint32_t tmem_slot;
+    __shared__ uint32_t tab_s[16];  // fp16 (hi | lo << 16) of every code (3- and 4-bit codes)
+    constexpr int kStageBytes = kTile * 16 * B;
+
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* hmat = smem;
+    uint8_t* ring = smem + kHBytes;
+    uint8_t* stage_out = ring + kStagesDq * kStageBytes;  // 2 x OutTile (1024-aligned)
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // codewords c_k 2^cs = hi_k + lo_k in fp16
+    float cmax = 0.0f;
+#pragma unroll
+    for (int k = 0; k < L; ++k) cmax = fmaxf(cmax, fabsf(__ldg(codebook + k)));
+    const int cs = (cmax > 0.0f) ? (13 - ilogbf(cmax)) : 0;
+    uint32_t hl[4], hh[4], ll[4], lh[4];  // bytes of hi / lo for codes 0..3
+    uint32_t th_lo = 0, th_hi = 0, tl_lo = 0, tl_hi = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float x = ldexpf(__ldg(codebook + (k < L ? k : L - 1)), cs);
+        const __half h = __float2half_rn(x);
+        const __half l = __float2half_rn(x - __half2float(h));
+        hl[k] = __half_as_ushort(h) & 0xffu;
+        hh[k] = __half_as_ushort(h) >> 8;
+        ll[k] = __half_as_ushort(l) & 0xffu;
+        lh[k] = __half_as_ushort(l) >> 8;
+        th_lo |= hl[k] << (8 * k);
+        th_hi |= hh[k] << (8 * k);
+        tl_lo |= ll[k] << (8 * k);
+        tl_hi |= lh[k] << (8 * k);
+    }
+    if (threadIdx.x < 16) {
+        const float x = ldexpf(__ldg(codebook + (threadIdx.x < L ? threadIdx.x : L - 1)), cs);
+        const __half h = __float2half_rn(x);
+        const __half l = __float2half_rn(x - __half2float(h));
+        tab_s[threadIdx.x] = static_cast<uint32_t>(__half_as_ushort(h)) |
+                             (static_cast<uint32_t>(__half_as_ushort(l)) << 16);
+    }
+    const float inv_scale = ldexpf(1.0f, -cs) * kInvSqrt128;
+
+    // B operand: row n, column k = H_int[n][e(k)] (fp16 +-1), K-major, 128-byte swizzle
+    for (int item = threadIdx.x; item < kTile * 16; item += kDqThreads) {
+        const int n = item >> 4, c16 = item & 15;
+        uint32_t w4[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const int k0 = c16 * 8 + 2 * p;
+            const uint32_t lo = (__popc(n & elem_of_col<B>(k0)) & 1) ? 0xBC00u : 0x3C00u;
+            const uint32_t hi = (__popc(n & elem_of_col<B>(k0 + 1)) & 1) ? 0xBC00u : 0x3C00u;
+            w4[p] = lo | (hi << 16);
+        }
+        const int half = c16 >> 3, kl = (c16 & 7);
+        *reinterpret_cast<uint4*>(hmat + half * kHHalf + n * 128 + ((kl ^ (n & 7)) << 4)) =
+            make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
+    fence_proxy_async_smem();
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStagesDq; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 4);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&afull_bar[a], 4);
+            mbar_init(&dfull_bar[a], 1);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(&tmem_slot, kTmemColsDq);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = tmem_slot;
+
+    if (warp == 0) {
+        // ---------------- bulk-copy producer ----------------
+        if (lane == 0) {
+            int i = 0;
+            for (long long t = blockIdx.x; t < sh.tiles; t += gridDim.x, ++i) {
+                const int st = i % kStagesDq;
+                if (!mbar_wait(&empty_bar[st], ((i / kStagesDq) & 1) ^ 1, status)) break;
+                const long long g0 = t * kTile;
+                const long long n = sh.total - g0 < kTile ? sh.total - g0 : kTile;
+                const uint32_t bytes = static_cast<uint32_t>(n) * (16 * B);
+                mbar_arrive_expect_tx(&full_bar[st], bytes);
+                bulk_load(ring + st * kStageBytes, packed + g0 * (16 * B), bytes, &full_bar[st]);
+            }
+            for (int k = 0; k < kStagesDq && k < i; ++k) {
+                const int ii = i - 1 - k;
+                mbar_wait(&empty_bar[ii % kStagesDq], (ii / kStagesDq) & 1, status);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            int i = 0;
+            for (long long t = blockIdx.x; t < sh.tiles; t += gridDim.x, ++i) {
+                const int e = i & 1;
+                if (!mbar_wait(&afull_bar[e], (i >> 1) & 1, status)) break;
+                tc_fence_after();
+                const uint32_t a_hi = tbase + e * kSlotCols, a_lo = a_hi + 64, d = a_hi + 128;
+                const uint32_t b_base = smem_u32(hmat);
+#pragma unroll
+                for (int k = 0; k < kTile / 16; ++k)
+                    mma_f16_tmem_a(d, a_hi + 8 * k,
+                                   smem_desc_sw128(b_base + (k >> 2) * kHHalf + (k & 3) * 32), kIdescDq,
+                                   k > 0);
+#pragma unroll
+                for (int k = 0; k < kTile / 16; ++k)
+                    mma_f16_tmem_a(d, a_lo + 8 * k,
+                                   smem_desc_sw128(b_base + (k >> 2) * kHHalf + (k & 3) * 32), kIdescDq,
+                                   true);
+                mma_commit(&dfull_bar[e]);
+            }
+        }
+    } else {
+        // ---------------- decode + epilogue ----------------
+        const int e = (warp - 2) >> 2;
+        const int quad = warp & 3;
+        const int m = quad * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+        const uint32_t a_hi = tbase + lane_off + e * kSlotCols, a_lo = a_hi + 64, d = a_hi + 128;
+        int i = e;
+        for (long long t = blockIdx.x + static_cast<long long>(e) * gridDim.x; t < sh.tiles;
+             t += 2LL * gridDim.x, i += 2) {
+            const int st = i % kStagesDq;
+            // the group's four warps decide together whether to go on
+            if (!named_barrier_and(1 + e, 128, mbar_wait(&full_bar[st], (i / kStagesDq) & 1, status))) break;
+            const long long gid = t * kTile + m;
+            const bool valid = gid < sh.total;
+            uint32_t wd[4 * B];
+            {
+                const uint4* src = reinterpret_cast<const uint4*>(ring + st * kStageBytes + m * (16 * B));
+#pragma unroll
+                for (int v = 0; v < B; ++v) {
+                    const uint4 u = valid ? src[v] : make_uint4(0, 0, 0, 0);
+                    wd[4 * v + 0] = u.x;
+                    wd[4 * v + 1] = u.y;
+                    wd[4 * v + 2] = u.z;
+                    wd[4 * v + 3] = u.w;
+                }
+            }
+            const float nrm = valid ? __half2float(__ushort_as_half(__ldg(norms + gid))) : 0.0f;
+
+            // A planes: 64 columns each, written 32 at a time
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t rh[32], rl[32];
+                if constexpr (B == 2) {
+#pragma unroll
+                    for (int ww = 0; ww < 4; ++ww) {
+                        const uint32_t word = wd[4 * half + ww];
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) {
+                            const uint32_t sw = (word >> (2 * p)) & 0x03030303u;
+                            const uint32_t s0 = sw * 0x11u + 0x4040u;
+                            const uint32_t s1 = mad_hi(sw, 0x110000u, 0x4040u);
+                            const int col = 8 * ww + 2 * p;  // within this 32-column half
+                            rh[col] = prmt(th_lo, th_hi, s0);
+                            rh[col + 1] = prmt(th_lo, th_hi, s1);
+                            rl[col] = prmt(tl_lo, tl_hi, s0);
+                            rl[col + 1] = prmt(tl_lo, tl_hi, s1);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const int e0 = 64 * half + 2 * c;  // elements e0, e0 + 1
+                        uint32_t code[2];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int bit = B * (e0 + u);
+                            const uint32_t lo = wd[bit >> 5];
+                            const uint32_t hi = ((bit >> 5) + 1 < 4 * B) ? wd[(bit >> 5) + 1] : 0u;
+                            uint32_t cd = __funnelshift_r(lo, hi, bit & 31) & ((1u << B) - 1u);
+                            code[u] = cd < static_cast<uint32_t>(L) ? cd : static_cast<uint32_t>(L - 1);
+                        }
+                        const uint32_t t0 = tab_s[code[0]], t1 = tab_s[code[1]];
+                        rh[c] = prmt(t0, t1, 0x5410u);
+                        rl[c] = prmt(t0, t1, 0x7632u);
+                    }
+                }
+                tmem_st32(a_hi + 32 * half, rh);
+                tmem_st32(a_lo + 32 * half, rl);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            // the stage's words are consumed (decoded); order these generic reads before the
+            // producer's next bulk write into the stage
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&empty_bar[st]);
+                mbar_arrive(&afull_bar[e]);
+            }
+
+            const bool leader = (warp == 2 + 4 * e) && lane == 0;
+            bool ok = mbar_wait(&dfull_bar[e], (i >> 1) & 1, status);
+            // before the staging tile is rewritten, this group's previous stores have read it
+            if (sh.flat && leader) bulk_wait_read0();
+            if (!named_barrier_and(1 + e, 128, ok)) break;
+            tc_fence_after();
+            const float scale = nrm * inv_scale;
+            constexpr int kPer = kBF16 ? 8 : 4;  // values per 16-byte chunk
+            if (sh.flat) {
+                // stage the tile in shared memory, then one tensor-map store per box
+                uint8_t* so = stage_out + e * OutTile<kBF16>::kBytes;
+#pragma unroll
+                for (int c = 0; c < kTile / 32; ++c) {
+                    float v[32];
+                    tmem_ld32(d + 32 * c, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int q = 0; q < 32 / kPer; ++q) {
+                        const int off = q * kPer;
+                        uint4 o;
+                        if constexpr (kBF16) {
+                            o.x = pack_bf16x2(v[off + 0] * scale, v[off + 1] * scale);
+                            o.y = pack_bf16x2(v[off + 2] * scale, v[off + 3] * scale);
+                            o.z = pack_bf16x2(v[off + 4] * scale, v[off + 5] * scale);
+                            o.w = pack_bf16x2(v[off + 6] * scale, v[off + 7] * scale);
+                        } else {
+                            o.x = __float_as_uint(v[off + 0] * scale);
+                            o.y = __float_as_uint(v[off + 1] * scale);
+                            o.z = __float_as_uint(v[off + 2] * scale);
+                            o.w = __float_as_uint(v[off + 3] * scale);
+                        }
+                        *reinterpret_cast<uint4*>(so + OutTile<kBF16>::chunk_offset(m, (32 * c + off) / kPer)) = o;
+                    }
+                }
+                fence_proxy_async_smem();
+                named_barrier(1 + e, 128);
+                if (leader) {
+#pragma unroll
+                    for (int b = 0; b < OutTile<kBF16>::kBoxes; ++b)
+                        tma_store_2d(&omap, b * OutTile<kBF16>::kPerBox, static_cast<int>(t * kTile),
+                                     so + b * OutTile<kBF16>::kBoxBytes);
+                    bulk_commit();
+                }
+            } else {
+                const long long row = gid / sh.G, j = gid - (gid / sh.G) * sh.G;
+                const long long base = row * sh.cols + j * kTile;
+#pragma unroll
+                for (int c = 0; c < kTile / 32; ++c) {
+                    float v[32];
+                    tmem_ld32(d + 32 * c, v);
+                    tmem_ld_wait();
+                    if (!valid) continue;
+#pragma unroll
+                    for (int q = 0; q < 32 / kPer; ++q) {
+                        const int off = q * kPer;
+                        if (j * kTile + 32 * c + off < sh.cols)
+                            store_chunk<kBF16>(out, base + 32 * c + off, v, off, scale);
+                    }
+                }
+            }
+        }
+        if (sh.flat && (warp == 2 + 4 * e) && lane == 0) bulk_wait0();  // stores done before exit
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tbase, kTmemColsDq);
+    }
+}
+
+template <int B, int L, bool kBF16>
+cudaError_t launch_dq(const uint8_t* packed, const uint16_t* norms, const DqShape& ds,
+                      const float* cb, void* out, unsigned* status, cudaStream_t st) {
+    const int smem = kHBytes + kStagesDq * kTile * 16 * B + 2 * OutTile<kBF16>::kBytes + 1024;
+    CUtensorMap omap;
+    std::memset(&omap, 0, sizeof(omap));
+    if (ds.flat) {
+        // the output viewed as [groups x 128] values, boxes of 128 bytes x 128 rows
+        const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(kTile), static_cast<cuuint64_t>(ds.total)};
+        const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(kTile) * (kBF16 ? 2 : 4)};
+        const cuuint32_t box[2] = {static_cast<cuuint32_t>(OutTile<kBF16>::kPerBox), kTile};
+        const cuuint32_t estride[2] = {1, 1};
+        EncodeTiledFn enc = tensor_map_encoder();
+        if (enc == nullptr) return cudaErrorNotSupported;
+        const CUresult r = enc(&omap, kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                               2, out, gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    }
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    static unsigned long long configured = 0;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(configured & bit)) {
+        e = cudaFuncSetAttribute(dequantize_tc_kernel<B, L, kBF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        configured |= bit;
+    }
+    const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(ds.tiles, sm_count())));
+    dequantize_tc_kernel<B, L, kBF16><<<grid, kDqThreads, smem, st>>>(packed, norms, ds, cb, out, status, omap);
+    return cudaGetLastError();
+}
+
+template <int B, int L>
+cudaError_t launch_dq_dtype(int out_dtype, const uint8_t* packed, const uint16_t* norms,
+                            const DqShape& ds, const float* cb, void* out, unsigned* status,
+                            cudaStream_t st) {
+    if (out_dtype == CQ_BF16) return launch_dq<B, L, true>(packed, norms, ds, cb, out, status, st);
+    return launch_dq<B, L, false>(packed, norms, ds, cb, out, status, st);
+}
+
+}  // namespace
+
+bool dequantize_tc_supported(int out_dtype, const Shape& sh) {
+    if (sh.cols % (out_dtype == CQ_BF16 ? 8 : 4) != 0) return false;
+    if (sh.cols % kTile == 0 && (sh.total_groups >= (1LL << 31) || tensor_map_encoder() == nullptr)) return false;
+    return true;
+}
+
+cudaError_t launch_dequantize_tc(const uint8_t* packed, const uint16_t* norms, const Shape& sh,
+                                 int bits, const float* codebook, void* out, int out_dtype,
+                                 unsigned* status, cudaStream_t stream) {
+    DqShape ds;
+    ds.total = sh.total_groups;
+    ds.cols = sh.cols;
+    ds.G = sh.groups_per_row;
+    ds.tiles = (sh.total_groups + kTile - 1) / kTile;
+    ds.flat = sh.cols % kTile == 0;
+    switch (bits) {
+        case CQ_BITS_TERNARY: return launch_dq_dtype<2, 3>(out_dtype, packed, norms, ds, codebook, out, status, stream);
+        case 2: return launch_dq_dtype<2, 4>(out_dtype, packed, norms, ds, codebook, out, status, stream);
+        case 3: return launch_dq_dtype<3, 8>(out_dtype, packed, norms, ds, codebook, out, status, stream);
+        default: return launch_dq_dtype<4, 16>(out_dtype, packed, norms, ds, codebook, out, status, stream);
+    }
+}
+
+}  // namespace cq

@@ -4,6 +4,7 @@
 #include <cstddef>
 #include <cstdint>
 
+#include <cuda.h>  // CUtensorMap and its enums (types only; no libcuda link)
 #include <cuda_runtime.h>
 
 #include "cq.h"
@@ -28,6 +29,14 @@ struct Shape {
 };
 
 // Kernel launchers (one per file).  All return cudaSuccess or the launch error.
+// cuTensorMapEncodeTiled, looked up once through the runtime's driver entry point (nullptr
+// when unavailable).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn tensor_map_encoder();
+
 // Device-wide status word of the current device (bit 0: a bounded wait inside a kernel gave
 // up).  Returns nullptr if the symbol address cannot be obtained.
 unsigned* device_status_ptr();
@@ -41,6 +50,12 @@ bool quantize_tc_supported(int w_dtype, const Shape& s);
 cudaError_t launch_quantize_tc(const void* w, const Shape& s, int bits, const float* codebook,
                                uint8_t* packed, uint16_t* norms, unsigned* status,
                                cudaStream_t stream);
+
+// Tensor-core dequantiser (cq_dequantize_tc.cu): rows of the output start on 16 bytes.
+bool dequantize_tc_supported(int out_dtype, const Shape& s);
+cudaError_t launch_dequantize_tc(const uint8_t* packed, const uint16_t* norms, const Shape& s,
+                                 int bits, const float* codebook, void* out, int out_dtype,
+                                 unsigned* status, cudaStream_t stream);
 
 cudaError_t launch_quantize(const void* w, int w_dtype, const Shape& s, int bits,
                             const float* codebook, uint8_t* packed, uint16_t* norms,

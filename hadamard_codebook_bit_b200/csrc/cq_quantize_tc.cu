@@ -26,7 +26,6 @@
 // cols % 128 == 0 the whole matrix is viewed as [groups x 128] (G_eff = 1), so one tile is
 // 128 consecutive groups and the packed output of a tile is one contiguous block.
 #include <algorithm>
-#include <mutex>
 
 #include "cq_device.cuh"
 #include "cq_internal.h"
@@ -293,25 +292,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
 }
 
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
-using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
-                              CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
-                              CUtensorMapFloatOOBfill);
-
-EncodeFn encode_fn() {
-    static EncodeFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeFn>(p);
-    });
-    return fn;
-}
-
 template <int B, int L>
 cudaError_t launch_tc(const CUtensorMap& map, const TcShape& ts, const float* cb, uint8_t* packed,
                       uint16_t* norms, unsigned* status, cudaStream_t st) {
@@ -338,7 +318,7 @@ bool quantize_tc_supported(int w_dtype, const Shape& sh) {
     const bool flat = sh.cols % kTile == 0;
     const long long r_eff = flat ? sh.total_groups : sh.rows;
     if (r_eff >= (1LL << 31)) return false;
-    return encode_fn() != nullptr;
+    return tensor_map_encoder() != nullptr;
 }
 
 cudaError_t launch_quantize_tc(const void* w, const Shape& sh, int bits, const float* codebook,
@@ -357,7 +337,7 @@ cudaError_t launch_quantize_tc(const void* w, const Shape& sh, int bits, const f
     const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(c_eff) * 2};
     const cuuint32_t box[2] = {64, kTile};
     const cuuint32_t estride[2] = {1, 1};
-    const CUresult r = encode_fn()(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(w), gdim,
+    const CUresult r = tensor_map_encoder()(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(w), gdim,
                                    gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
                                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
