@@ -12,20 +12,24 @@
 //   tensor-core B operand; the exponents go to an fp32 table.  Block 0 also writes the
 //   codeword table (fp16, one exact power-of-two scale) used by step 2.
 //
-// Step 2 (gemv_mma_kernel, launched as a programmatic dependent of step 1): a 4-warp block
-// owns 16 output rows.  The packed blocks of those rows are copied to shared memory with
-// cp.async before anything else (the whole tile's loads are in flight at once), then each
-// warp takes every fourth group: eight m16n8k16 fp16 MMAs per group (A = decoded codewords
-// of 16 rows x 16 weights, B = x~ of 16 weights x 8 columns, fp32 accumulate), folded into
-// fp32 totals as  total += n_rj * 2^e_bj * acc.  The warps' totals are summed in a fixed
-// order, so the output is deterministic.
+// Step 2 (gemv_split_kernel, launched as a programmatic dependent of step 1): a block of S
+// warps owns 16 output rows; warp w takes a contiguous chunk of about G / S groups, S chosen
+// so that all row blocks are resident at once.  Per group a lane reads
+// its 32 codes of rows g and g + 8 straight from global memory (one coalesced 8/12/16-byte
+// load per row, four groups in flight at once), decodes them into fp16 A fragments and issues
+// eight m16n8k16 fp16 MMAs (A = codewords of 16 rows x 16 weights, B = x~ of 16 weights x 8
+// columns, fp32 accumulate), folded into fp32 totals as  total += n_rj * 2^e_bj * acc.  The S
+// warps' totals are summed in a fixed order, so the output is deterministic.
 //
 // K order inside a group.  The MMA contracts over the 16 weights of a k-step in any order
-// as long as A and B agree.  Lane (g, t) = (lane / 4, lane % 4) in k-step s takes the
-// weights  e = 16 w + 4 q + p,  q = 0..3,  with  w = t + 4 (s / 4)  and  p = s % 4:  the
-// four codes sitting at bit 2p of the four bytes of packed word w.  For 2-bit codes the
-// decode is then an (immediate) shift, a mask, two integer multiply-adds that form
-// byte-permute selectors, and two PRMTs from a 4-entry fp16 table held in two registers.
+// as long as A and B agree.  Lane (g, t) = (lane / 4, lane % 4) holds codes 32 t .. 32 t + 31
+// of each of its rows; in k-step s its four weights q = 0..3 (MMA k = 2t, 2t+1, 2t+8, 2t+9) are
+//   2-bit:    e = 32 t + 16 (s / 4) + 4 q + s % 4  (the codes at bit 2 (s % 4) of the four
+//             bytes of the lane's word s / 4: decoded with a shift, a mask, two integer
+//             multiply-adds that form byte-permute selectors and two PRMTs from a 4-entry
+//             fp16 table held in two registers);
+//   3/4-bit:  e = 32 t + 4 s + q  (four adjacent codes: one 12- or 16-bit field, spread to
+//             nibble selectors, looked up with byte permutes in 8 / 16-entry byte tables).
 #include <algorithm>
 
 #include "cq_device.cuh"
@@ -38,12 +42,10 @@ using namespace dev;
 
 constexpr int kRotThreads = 256;  // 8 warps = 8 batch columns
 constexpr int kRowsPerBlock = 16;
-constexpr int kWarps = 4;
-constexpr int kThreads = 32 * kWarps;
 constexpr int kBatchCols = 8;     // MMA N: batch columns, zero padded
 constexpr int kXEntry = 8;        // bytes of B fragment per lane per k-step (4 fp16)
 
-// Workspace: [G][8 k-steps][32 lanes] of 4 fp16 | fp32 exponents [G][8] | codeword table.
+// Workspace: [G][4 k-step pairs][32 lanes] of 8 fp16 | fp32 exponents [G][8] | codeword table.
 size_t frag_bytes(long long G) { return static_cast<size_t>(G) * 8 * 32 * kXEntry; }
 size_t scale_bytes(long long G) { return static_cast<size_t>(G) * kBatchCols * sizeof(float); }
 
@@ -66,6 +68,11 @@ __device__ __forceinline__ uint32_t mad_hi(uint32_t a, uint32_t b, uint32_t c) {
     return d;
 }
 
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+    return static_cast<uint32_t>(__half_as_ushort(__float2half_rn(lo))) |
+           (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(hi))) << 16);
+}
+
 __device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                           uint32_t a3, uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -79,7 +86,7 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a
 // step 1: rotate the activations into fragment order (+ codeword table)
 // ---------------------------------------------------------------------------------------
 
-template <int L>
+template <int B, int L>
 __global__ void __launch_bounds__(kRotThreads)
     rotate_x_kernel(const uint16_t* __restrict__ x, long long cols, long long G, int batch,
                     const float* __restrict__ codebook, __half* __restrict__ xfrag,
@@ -141,14 +148,21 @@ __global__ void __launch_bounds__(kRotThreads)
     const int e = (mx > 0.0f) ? (ilogbf(mx) - 13) : 0;
     const float down = ldexpf(1.0f, -e);
     if (lane == 0) xscale[j * kBatchCols + b] = ldexpf(1.0f, e);
-    // element el = 4 lane + i = 16 w + 4 q + p  ->  k-step s = p + 4 (w / 4), lane 4 b + w % 4,
-    // half q of the lane's 4-value entry
-    const int w = lane >> 2, q = lane & 3;
-    const int t = w & 3, shi = w >> 2;
+    // element e = 4 lane + i  ->  (k-step s, lane 4 b + t, half q); entry layout
+    // [j][s / 2][lane][8 halves], halves 4 (s % 2) + q
+    const int t = lane >> 3;
+    if constexpr (B == 2) {
+        const int wsel = (lane >> 2) & 1, q = lane & 3;
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-        const int s = p + 4 * shi;
-        xfrag[((j * 8 + s) * 32 + 4 * b + t) * 4 + q] = __float2half_rn(v[p] * down);
+        for (int p = 0; p < 4; ++p) {
+            const int s = 4 * wsel + p;
+            xfrag[((j * 4 + (s >> 1)) * 32 + 4 * b + t) * 8 + 4 * (s & 1) + q] = __float2half_rn(v[p] * down);
+        }
+    } else {
+        const int s = lane & 7;
+        const uint32_t h01 = pack_half2(v[0] * down, v[1] * down), h23 = pack_half2(v[2] * down, v[3] * down);
+        *reinterpret_cast<uint2*>(xfrag + ((j * 4 + (s >> 1)) * 32 + 4 * b + t) * 8 + 4 * (s & 1)) =
+            make_uint2(h01, h23);
     }
 }
 
@@ -156,286 +170,315 @@ __global__ void __launch_bounds__(kRotThreads)
 // step 2: streaming tensor-core GEMV
 // ---------------------------------------------------------------------------------------
 
-__device__ __forceinline__ long long min64(long long a, long long b) { return a < b ? a : b; }
-
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-// Groups are staged in chunks of kChunk; a stage holds 16 rows x kChunk blocks, each row
-// padded by 16 bytes so the eight rows a warp reads at once fall in different banks.
-constexpr int kChunk = 32;
-constexpr int kStages = 4;
-
+// Codes of one lane for one group row: words 2t, 2t+1 (2-bit), 3t..3t+2 (3-bit), 4t..4t+3.
 template <int B>
-struct Stage {
-    static constexpr int kRowBytes = kChunk * 16 * B + 16;
-    static constexpr int kBytes = kRowsPerBlock * kRowBytes;
+struct Seg {
+    uint32_t w[B];
 };
 
 template <int B>
-__device__ __forceinline__ void issue_chunk(const uint8_t* __restrict__ packed, long long rows,
-                                            long long G, long long r0, long long j0, int len,
-                                            uint8_t* stage) {
-    constexpr int kFullPieces = kChunk * B;  // 16-byte pieces per row of a full chunk
-    if (len == kChunk) {
-        for (int i = threadIdx.x; i < kRowsPerBlock * kFullPieces; i += kThreads) {
-            const int r = i / kFullPieces, p = i % kFullPieces;
-            if (r0 + r < rows)
-                cp_async16(stage + r * Stage<B>::kRowBytes + 16 * p,
-                           packed + ((r0 + r) * G + j0) * (16 * B) + 16 * p);
-        }
-    } else {
-        const int pieces = len * B;
-        for (int i = threadIdx.x; i < kRowsPerBlock * pieces; i += kThreads) {
-            const int r = i / pieces, p = i - r * pieces;
-            if (r0 + r < rows)
-                cp_async16(stage + r * Stage<B>::kRowBytes + 16 * p,
-                           packed + ((r0 + r) * G + j0) * (16 * B) + 16 * p);
-        }
-    }
-}
-
-// The 16 B-bit codes lane t uses from one group row, for the halves h = 0 (k-steps 0-3) and
-// h = 1 (k-steps 4-7): bits [16 B w0, 16 B w0 + 16 B) of the block with w0 = t + 4 h.
-template <int B>
-struct RowCodes {
-    uint32_t seg[2][(B + 1) / 2];  // 1 word per half for B = 2, 2 words for B = 3, 4
-};
-
-template <int B>
-__device__ __forceinline__ void load_codes(const uint8_t* row, int t, RowCodes<B>& rc) {
-    const uint32_t* wd = reinterpret_cast<const uint32_t*>(row);
+__device__ __forceinline__ Seg<B> load_seg(const uint8_t* __restrict__ blk, int t, bool ok) {
+    Seg<B> r;
+    if (!ok) {
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int w0 = t + 4 * h;
-        if constexpr (B == 2) {
-            rc.seg[h][0] = wd[w0];
-        } else if constexpr (B == 4) {
-            rc.seg[h][0] = wd[2 * w0];
-            rc.seg[h][1] = wd[2 * w0 + 1];
-        } else {
-            // 48 bits at bit 48 w0: three words from word 3 w0 / 2, shifted by 16 (w0 & 1)
-            const int wi = (3 * w0) >> 1;
-            const uint32_t a = wd[wi], b = wd[wi + 1], c = wd[wi + 2];
-            const uint32_t sh = 16u * (w0 & 1);
-            rc.seg[h][0] = __funnelshift_r(a, b, sh);
-            rc.seg[h][1] = __funnelshift_r(b, c, sh);
-        }
+        for (int i = 0; i < B; ++i) r.w[i] = 0u;
+        return r;
     }
-}
-
-// A-fragment pair of one row in k-step s: (c[e0], c[e1]) and (c[e2], c[e3]).
-template <int B>
-__device__ __forceinline__ void decode(const RowCodes<B>& rc, int s, uint32_t tlo, uint32_t thi,
-                                       const uint16_t* __restrict__ tab, uint32_t& r0, uint32_t& r1) {
-    const int h = s >> 2, p = s & 3;
     if constexpr (B == 2) {
-        const uint32_t sw = (rc.seg[h][0] >> (2 * p)) & 0x03030303u;  // code q in byte q
-        r0 = prmt(tlo, thi, sw * 0x11u + 0x4040u);                  // selectors of codes 0, 1
-        r1 = prmt(tlo, thi, mad_hi(sw, 0x110000u, 0x4040u));        // selectors of codes 2, 3
+        asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
+                     : "=r"(r.w[0]), "=r"(r.w[1])
+                     : "l"(blk + 8 * t));
+    } else if constexpr (B == 4) {
+        const uint4 v = ld_stream16(blk + 16 * t);
+        r.w[0] = v.x;
+        r.w[1] = v.y;
+        r.w[2] = v.z;
+        r.w[3] = v.w;
     } else {
-        uint32_t code[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int bit = B * (4 * q + p);  // within the 16 B-bit segment
-            const uint32_t lo = rc.seg[h][bit >> 5];
-            const uint32_t hi = ((bit >> 5) + 1 < (B + 1) / 2) ? rc.seg[h][(bit >> 5) + 1] : 0u;
-            code[q] = __funnelshift_r(lo, hi, bit & 31) & ((1u << B) - 1u);
-        }
-        r0 = static_cast<uint32_t>(tab[code[0]]) | (static_cast<uint32_t>(tab[code[1]]) << 16);
-        r1 = static_cast<uint32_t>(tab[code[2]]) | (static_cast<uint32_t>(tab[code[3]]) << 16);
+        for (int i = 0; i < 3; ++i)
+            asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r.w[i]) : "l"(blk + 12 * t + 4 * i));
+    }
+    return r;
+}
+
+// Byte tables of the fp16 codewords: lo[k] / hi[k] hold the low / high bytes of codes
+// 4k..4k+3.  The 2-bit decode uses lo[0], hi[0] only.
+struct ByteTables {
+    uint32_t lo[4], hi[4];
+};
+
+// x >> n with the shift on the integer multiply-add unit (n > 0), keeping the ALU free for
+// the masks and byte permutes
+template <int N>
+__device__ __forceinline__ uint32_t shr_mul(uint32_t x) {
+    if constexpr (N == 0) {
+        return x;
+    } else {
+        return mad_hi(x, 1u << (32 - N), 0u);
     }
 }
 
-template <int B, int NST>
-__global__ void __launch_bounds__(kThreads, 8)
-    gemv_mma_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ norms,
-                    long long rows, long long G, const uint2* __restrict__ xfrag,
-                    const float* __restrict__ xscale, const CodeTable* __restrict__ table,
-                    int batch, float* __restrict__ y) {
-    extern __shared__ __align__(16) uint8_t smem[];  // NST stages, then NST norm tiles
-    float* nrm_s = reinterpret_cast<float*>(smem + NST * Stage<B>::kBytes);
-    __shared__ float4 red[kWarps][32];
-    __shared__ uint16_t tab_s[16];
-    constexpr int kNrm = kRowsPerBlock * kChunk;
-    constexpr int kNrmPerThread = kNrm / kThreads;
+// A-fragment registers of one row in k-step S: r0 = (c[k=2t], c[2t+1]), r1 = (c[2t+8], c[2t+9]).
+template <int B, int S>
+__device__ __forceinline__ void decode(const Seg<B>& sg, const ByteTables& tb, uint32_t& r0, uint32_t& r1) {
+    if constexpr (B == 2) {
+        const uint32_t sw = shr_mul<2 * (S & 3)>(sg.w[S >> 2]) & 0x03030303u;  // code q in byte q
+        r0 = prmt(tb.lo[0], tb.hi[0], sw * 0x11u + 0x4040u);                 // codes q = 0, 1
+        r1 = prmt(tb.lo[0], tb.hi[0], mad_hi(sw, 0x110000u, 0x4040u));       // codes q = 2, 3
+    } else {
+        uint32_t sel, m = 0x3210u;
+        uint32_t lo4, hi4;
+        if constexpr (B == 4) {
+            const uint32_t f = (S & 1) ? (sg.w[S >> 1] >> 16) : sg.w[S >> 1];  // 4 codes in nibbles
+            sel = f & 0x7777u;
+            m |= (f >> 1) & 0x4444u;  // code >= 8: take the byte from the upper 8-entry half
+            lo4 = prmt(prmt(tb.lo[0], tb.lo[1], sel), prmt(tb.lo[2], tb.lo[3], sel), m);
+            hi4 = prmt(prmt(tb.hi[0], tb.hi[1], sel), prmt(tb.hi[2], tb.hi[3], sel), m);
+        } else {
+            constexpr int kBit = 12 * S;  // four 3-bit codes at bits 12 S .. 12 S + 11
+            uint32_t f;
+            if constexpr ((kBit & 31) + 12 <= 32) {
+                f = sg.w[kBit >> 5] >> (kBit & 31);
+            } else {
+                f = __funnelshift_r(sg.w[kBit >> 5], sg.w[(kBit >> 5) + 1], kBit & 31);
+            }
+            sel = (f & 0x7u) | ((f << 1) & 0x70u) | ((f << 2) & 0x700u) | ((f << 3) & 0x7000u);
+            lo4 = prmt(tb.lo[0], tb.lo[1], sel);
+            hi4 = prmt(tb.hi[0], tb.hi[1], sel);
+        }
+        r0 = prmt(lo4, hi4, 0x5140u);
+        r1 = prmt(lo4, hi4, 0x7362u);
+    }
+}
 
+__device__ __forceinline__ uint4 ld_v4_volatile(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// Byte tables and scale from the codeword table step 1 wrote (volatile loads: see load_bfrag).
+template <int B>
+__device__ __forceinline__ void load_tables(const CodeTable* table, ByteTables& tb, float& inv_scale) {
+    const uint4 head = ld_v4_volatile(table);  // lo, hi, inv_scale, pad
+    inv_scale = __uint_as_float(head.z);
+    if constexpr (B == 2) {
+        tb.lo[0] = head.x;
+        tb.hi[0] = head.y;
+    } else {
+        const uint4 h0 = ld_v4_volatile(reinterpret_cast<const uint8_t*>(table) + 16);  // h[0..7]
+        const uint4 h1 = ld_v4_volatile(reinterpret_cast<const uint8_t*>(table) + 32);  // h[8..15]
+        const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            // codes 4k..4k+3 = words 2k, 2k+1 (two fp16 each)
+            const uint32_t a = hw[2 * k], c = hw[2 * k + 1];
+            tb.lo[k] = prmt(a, c, 0x6420u);  // low bytes
+            tb.hi[k] = prmt(a, c, 0x7531u);  // high bytes
+        }
+    }
+}
+
+constexpr int kMaxSplit = 16;  // warps per block
+// groups per warp in flight (fewer for the wider 3/4-bit code words)
+template <int B>
+constexpr int kDepth = B == 2 ? 8 : 4;
+
+// B fragments of one group (four k-step pairs); lanes holding padding columns skip the loads
+// and keep the zeros they were initialised with.  Everything step 1 writes is read with
+// volatile asm so that no read can be moved above the griddepcontrol.wait.
+__device__ __forceinline__ void load_bfrag(const uint4* __restrict__ p, bool on, uint4 (&bf)[4]) {
+#pragma unroll
+    for (int sp = 0; sp < 4; ++sp)
+        asm volatile(
+            "{\n\t.reg .pred q;\n\t"
+            "setp.ne.u32 q, %4, 0;\n\t"
+            "@q ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%5];\n\t}"
+            : "+r"(bf[sp].x), "+r"(bf[sp].y), "+r"(bf[sp].z), "+r"(bf[sp].w)
+            : "r"(static_cast<uint32_t>(on)), "l"(p + sp * 32));
+}
+
+// One warp's walk over its chunk of groups for 16 rows (rows past the end read row 0 and are
+// dropped at the end, so no load is predicated on the row).
+template <int B>
+struct GemvWarp {
+    static constexpr int kBlk = 16 * B;
+    const uint8_t* pa;   // packed block of row g at the current group
+    const uint8_t* pb;   // ... row g + 8
+    const uint16_t* na;  // norms of row g at the current group
+    const uint16_t* nb;
+    const uint4* xf;     // B fragments of the current group, this lane
+    const float2* xs;    // exponents of the current group, columns 2t, 2t + 1
+    bool bcol;           // this lane holds a real batch column
+    int t;
+    ByteTables tb;
+    uint4 bf[4];
+    float tot[4];
+
+    // kDepth<B> groups (or the first n of them when !kFull): all loads first, then the math
+    template <bool kFull>
+    __device__ __forceinline__ void batch(int n) {
+        Seg<B> ca[kDepth<B>], cb[kDepth<B>];
+        float sa[kDepth<B>], sb[kDepth<B>];
+#pragma unroll
+        for (int u = 0; u < kDepth<B>; ++u) {
+            const bool on = kFull || u < n;
+            ca[u] = load_seg<B>(pa + u * kBlk, t, on);
+            cb[u] = load_seg<B>(pb + u * kBlk, t, on);
+            sa[u] = on ? __half2float(__ushort_as_half(__ldg(na + u))) : 0.0f;
+            sb[u] = on ? __half2float(__ushort_as_half(__ldg(nb + u))) : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < kDepth<B>; ++u) {
+            if (!kFull && u >= n) break;
+            load_bfrag(xf + u * 128, bcol, bf);
+            float2 x2;  // volatile: stays after the dependency wait
+            asm volatile("ld.global.nc.v2.f32 {%0, %1}, [%2];" : "=f"(x2.x), "=f"(x2.y) : "l"(xs + u * 4));
+            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            uint32_t a0, a1, a2, a3;
+#define CQ_KSTEP(SS, B0, B1)                   \
+    decode<B, SS>(ca[u], tb, a0, a2);          \
+    decode<B, SS>(cb[u], tb, a1, a3);          \
+    mma_16816(acc, a0, a1, a2, a3, B0, B1);
+            CQ_KSTEP(0, bf[0].x, bf[0].y)
+            CQ_KSTEP(1, bf[0].z, bf[0].w)
+            CQ_KSTEP(2, bf[1].x, bf[1].y)
+            CQ_KSTEP(3, bf[1].z, bf[1].w)
+            CQ_KSTEP(4, bf[2].x, bf[2].y)
+            CQ_KSTEP(5, bf[2].z, bf[2].w)
+            CQ_KSTEP(6, bf[3].x, bf[3].y)
+            CQ_KSTEP(7, bf[3].z, bf[3].w)
+#undef CQ_KSTEP
+            tot[0] = fmaf(sa[u] * x2.x, acc[0], tot[0]);
+            tot[1] = fmaf(sa[u] * x2.y, acc[1], tot[1]);
+            tot[2] = fmaf(sb[u] * x2.x, acc[2], tot[2]);
+            tot[3] = fmaf(sb[u] * x2.y, acc[3], tot[3]);
+        }
+        pa += kDepth<B> * kBlk;
+        pb += kDepth<B> * kBlk;
+        na += kDepth<B>;
+        nb += kDepth<B>;
+        xf += kDepth<B> * 128;
+        xs += kDepth<B> * 4;
+    }
+};
+
+template <int B>
+__global__ void __maxnreg__(96)
+    gemv_split_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ norms,
+                      long long rows, int G, const uint4* xfrag, const float2* xscale,
+                      const CodeTable* table, int batch, float* __restrict__ y) {
+    __shared__ float4 red[kMaxSplit][32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int S = static_cast<int>(blockDim.x >> 5);
     const int g = lane >> 2, t = lane & 3;
     const long long r0 = static_cast<long long>(blockIdx.x) * kRowsPerBlock;
     const long long ra = r0 + g, rb = r0 + g + 8;
     const bool oka = ra < rows, okb = rb < rows;
-    const long long nchunks = (G + kChunk - 1) / kChunk;
 
-    auto norm_at = [&](long long c, int i) -> float {  // i-th norm of chunk c ([row][jj])
-        const int r = i / kChunk, jj = i % kChunk;
-        const long long j = c * kChunk + jj;
-        return (c < nchunks && r0 + r < rows && j < G)
-                   ? __half2float(__ushort_as_half(__ldg(norms + (r0 + r) * G + j)))
-                   : 0.0f;
-    };
+    // this warp's groups: [jb, je)
+    const int chunk = (G + S - 1) / S;
+    const int jb = min(G, warp * chunk), je = min(G, jb + chunk);
 
-    // prologue (independent of step 1): weight copies, then norms
-    for (int c = 0; c < NST; ++c) {
-        if (c < nchunks) {
-            const long long j0 = c * kChunk;
-            issue_chunk<B>(packed, rows, G, r0, j0, static_cast<int>(min64(kChunk, G - j0)),
-                           smem + c * Stage<B>::kBytes);
-        }
-        cp_async_commit();
-    }
-    {
-        float tmp[NST * kNrmPerThread];
+    GemvWarp<B> st;
+    st.pa = packed + ((oka ? ra : 0) * G + jb) * GemvWarp<B>::kBlk;
+    st.pb = packed + ((okb ? rb : 0) * G + jb) * GemvWarp<B>::kBlk;
+    st.na = norms + (oka ? ra : 0) * G + jb;
+    st.nb = norms + (okb ? rb : 0) * G + jb;
+    st.xf = xfrag + static_cast<long long>(jb) * 128 + lane;
+    st.xs = xscale + static_cast<long long>(jb) * 4 + t;
+    st.bcol = g < batch;
+    st.t = t;
 #pragma unroll
-        for (int c = 0; c < NST; ++c)
-#pragma unroll
-            for (int q = 0; q < kNrmPerThread; ++q)
-                tmp[c * kNrmPerThread + q] = norm_at(c, threadIdx.x + q * kThreads);
-#pragma unroll
-        for (int c = 0; c < NST; ++c)
-#pragma unroll
-            for (int q = 0; q < kNrmPerThread; ++q)
-                nrm_s[c * kNrm + threadIdx.x + q * kThreads] = tmp[c * kNrmPerThread + q];
-    }
+    for (int sp = 0; sp < 4; ++sp) st.bf[sp] = make_uint4(0, 0, 0, 0);
+    st.tot[0] = st.tot[1] = st.tot[2] = st.tot[3] = 0.0f;
 
-    // the rotated activations and the codeword table come from step 1
+    // Nothing is read before the dependency wait: loads issued earlier by a programmatic
+    // dependent (even of buffers written by kernels that ran before step 1) returned stale
+    // data on this hardware.  The early launch still hides the launch latency.
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const uint32_t tlo = table->lo, thi = table->hi;
-    const float inv_scale = table->inv_scale;
-    if (B != 2 && threadIdx.x < 16) tab_s[threadIdx.x] = table->h[threadIdx.x];
+    float inv_scale;
+    load_tables<B>(table, st.tb, inv_scale);
 
-    float tot[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    for (long long c = 0; c < nchunks; ++c) {
-        const int st = static_cast<int>(c % NST);
-        cp_async_wait<NST - 1>();
+    int n = je - jb;
+    for (; n >= kDepth<B>; n -= kDepth<B>) st.template batch<true>(n);
+    if (n > 0) st.template batch<false>(n);
+
+    float4 a = make_float4(st.tot[0], st.tot[1], st.tot[2], st.tot[3]);
+    if (S > 1) {
+        red[warp][lane] = a;
         __syncthreads();
-        const long long j0 = c * kChunk;
-        const int len = static_cast<int>(min64(kChunk, G - j0));
-        const uint8_t* base = smem + st * Stage<B>::kBytes;
-        const float* nst = nrm_s + st * kNrm;
-        uint2 bf[8];
-        if (warp < len) {
-            const uint2* xf = xfrag + (j0 + warp) * 8 * 32 + lane;
-#pragma unroll
-            for (int s = 0; s < 8; ++s) bf[s] = __ldg(xf + s * 32);
-        }
-        for (int jj = warp; jj < len; jj += kWarps) {
-            uint2 bn[8];  // B fragments of this warp's next group, fetched during this one
-            const int jn = jj + kWarps;
-            if (jn < len) {
-                const uint2* xf = xfrag + (j0 + jn) * 8 * 32 + lane;
-#pragma unroll
-                for (int s = 0; s < 8; ++s) bn[s] = __ldg(xf + s * 32);
-            }
-            RowCodes<B> ca, cb;
-            load_codes<B>(base + g * Stage<B>::kRowBytes + jj * 16 * B, t, ca);
-            load_codes<B>(base + (g + 8) * Stage<B>::kRowBytes + jj * 16 * B, t, cb);
-            const long long j = j0 + jj;
-            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                uint32_t a0, a1, a2, a3;
-                decode<B>(ca, s, tlo, thi, tab_s, a0, a2);
-                decode<B>(cb, s, tlo, thi, tab_s, a1, a3);
-                mma_16816(acc, a0, a1, a2, a3, bf[s].x, bf[s].y);
-            }
-            const float sa = nst[g * kChunk + jj], sb = nst[(g + 8) * kChunk + jj];
-            const float x0 = __ldg(xscale + j * kBatchCols + 2 * t);
-            const float x1 = __ldg(xscale + j * kBatchCols + 2 * t + 1);
-            tot[0] = fmaf(sa * x0, acc[0], tot[0]);
-            tot[1] = fmaf(sa * x1, acc[1], tot[1]);
-            tot[2] = fmaf(sb * x0, acc[2], tot[2]);
-            tot[3] = fmaf(sb * x1, acc[3], tot[3]);
-#pragma unroll
-            for (int s = 0; s < 8; ++s) bf[s] = bn[s];
-        }
-        __syncthreads();  // stage st fully consumed
-        const long long cn = c + NST;
-        if (cn < nchunks) {
-            const long long jn = cn * kChunk;
-            issue_chunk<B>(packed, rows, G, r0, jn, static_cast<int>(min64(kChunk, G - jn)),
-                           smem + st * Stage<B>::kBytes);
-        }
-        cp_async_commit();
-        if (cn < nchunks) {
-            float tmp[kNrmPerThread];
-#pragma unroll
-            for (int q = 0; q < kNrmPerThread; ++q) tmp[q] = norm_at(cn, threadIdx.x + q * kThreads);
-#pragma unroll
-            for (int q = 0; q < kNrmPerThread; ++q) nrm_s[st * kNrm + threadIdx.x + q * kThreads] = tmp[q];
-        }
-    }
-    cp_async_wait<0>();
-    red[warp][lane] = make_float4(tot[0], tot[1], tot[2], tot[3]);
-    __syncthreads();
-    if (warp == 0) {
-        float4 a = red[0][lane];
-#pragma unroll
-        for (int w = 1; w < kWarps; ++w) {
+        if (warp != 0) return;
+        a = red[0][lane];
+        for (int w = 1; w < S; ++w) {
             const float4 b = red[w][lane];
             a.x += b.x;
             a.y += b.y;
             a.z += b.z;
             a.w += b.w;
         }
-        const float f = inv_scale * kInvSqrt128;
-        const int c0 = 2 * t, c1 = 2 * t + 1;
-        if (oka && c0 < batch) y[c0 * rows + ra] = a.x * f;
-        if (oka && c1 < batch) y[c1 * rows + ra] = a.y * f;
-        if (okb && c0 < batch) y[c0 * rows + rb] = a.z * f;
-        if (okb && c1 < batch) y[c1 * rows + rb] = a.w * f;
     }
+    const float f = inv_scale * kInvSqrt128;
+    const int c0 = 2 * t, c1 = 2 * t + 1;
+    if (oka && c0 < batch) y[c0 * rows + ra] = a.x * f;
+    if (oka && c1 < batch) y[c1 * rows + ra] = a.y * f;
+    if (okb && c0 < batch) y[c0 * rows + rb] = a.z * f;
+    if (okb && c1 < batch) y[c1 * rows + rb] = a.w * f;
 }
 
-template <int B, int NST>
-cudaError_t launch_gemv_cfg(const uint8_t* packed, const uint16_t* norms, const Shape& sh,
-                            const uint2* xfrag, const float* xscale, const CodeTable* table,
-                            int batch, float* y, cudaStream_t st) {
-    const long long blocks = (sh.rows + kRowsPerBlock - 1) / kRowsPerBlock;
-    const int smem = NST * (Stage<B>::kBytes + kRowsPerBlock * kChunk * static_cast<int>(sizeof(float)));
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    static unsigned long long configured = 0;  // one bit per device (function attributes are per device)
-    const unsigned long long bit = 1ull << (dev & 63);
-    if (!(configured & bit)) {
-        e = cudaFuncSetAttribute(gemv_mma_kernel<B, NST>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        configured |= bit;
+// Registers per thread of gemv_split_kernel<B> on the current device (queried once).
+template <int B>
+int gemv_regs() {
+    static int regs = 0;
+    if (regs == 0) {
+        cudaFuncAttributes fa;
+        regs = (cudaFuncGetAttributes(&fa, gemv_split_kernel<B>) == cudaSuccess && fa.numRegs > 0) ? fa.numRegs : 128;
     }
+    return regs;
+}
+
+// Warps per block.  The row blocks are spread over the SMs in one round when they fit:
+// every SM holds ceil(blocks / SMs) of them, and the split is the largest (up to 16 warps,
+// at least two groups a warp) for which that many blocks stay resident by registers.
+int gemv_split(long long blocks, long long G, int regs) {
+    const long long sms = sm_count();
+    const long long per_sm = (blocks + sms - 1) / sms;
+    int best = 1;
+    for (int s = 2; s <= kMaxSplit && 2LL * s <= G; ++s) {
+        const long long by_regs = 65536LL / (32LL * s * regs);
+        const long long by_warps = 64 / s;
+        if (std::min(by_regs, by_warps) >= per_sm) best = s;
+    }
+    return best;
+}
+
+template <int B>
+cudaError_t launch_gemv_bits(const uint8_t* packed, const uint16_t* norms, const Shape& sh,
+                             const uint4* xfrag, const float2* xscale, const CodeTable* table,
+                             int batch, float* y, cudaStream_t st) {
+    const long long blocks = (sh.rows + kRowsPerBlock - 1) / kRowsPerBlock;
+    const int split = gemv_split(blocks, sh.groups_per_row, gemv_regs<B>());
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(blocks));
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.blockDim = dim3(static_cast<unsigned>(32 * split));
+    cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemv_mma_kernel<B, NST>, packed, norms, sh.rows, sh.groups_per_row,
-                              xfrag, xscale, table, batch, y);
+    return cudaLaunchKernelEx(&cfg, gemv_split_kernel<B>, packed, norms, sh.rows,
+                              static_cast<int>(sh.groups_per_row), xfrag, xscale, table, batch, y);
 }
 
-template <int B>
-cudaError_t launch_gemv_bits(const uint8_t* packed, const uint16_t* norms, const Shape& sh,
-                             const uint2* xfrag, const float* xscale, const CodeTable* table,
-                             int batch, float* y, cudaStream_t st) {
-    const long long nchunks = (sh.groups_per_row + kChunk - 1) / kChunk;
-    if (nchunks <= 1) return launch_gemv_cfg<B, 1>(packed, norms, sh, xfrag, xscale, table, batch, y, st);
-    if (nchunks == 2) return launch_gemv_cfg<B, 2>(packed, norms, sh, xfrag, xscale, table, batch, y, st);
-    return launch_gemv_cfg<B, kStages>(packed, norms, sh, xfrag, xscale, table, batch, y, st);
-}
-
-template <int L>
+template <int B, int L>
 cudaError_t launch_rotate(const uint16_t* x, const Shape& sh, int batch, const float* codebook,
                           __half* xfrag, float* xscale, CodeTable* table, cudaStream_t st) {
-    rotate_x_kernel<L><<<static_cast<unsigned>(sh.groups_per_row), kRotThreads, 0, st>>>(
+    rotate_x_kernel<B, L><<<static_cast<unsigned>(sh.groups_per_row), kRotThreads, 0, st>>>(
         x, sh.cols, sh.groups_per_row, batch, codebook, xfrag, xscale, table);
     return cudaGetLastError();
 }
@@ -457,21 +500,22 @@ cudaError_t launch_dequant_gemv(const uint8_t* packed, const uint16_t* norms, co
     __half* xfrag = reinterpret_cast<__half*>(ws);
     float* xscale = reinterpret_cast<float*>(ws + frag_bytes(G));
     CodeTable* table = reinterpret_cast<CodeTable*>(ws + frag_bytes(G) + scale_bytes(G));
-    const uint2* xf = reinterpret_cast<const uint2*>(xfrag);
+    const uint4* xf = reinterpret_cast<const uint4*>(xfrag);
+    const float2* xs = reinterpret_cast<const float2*>(xscale);
     cudaError_t e;
     switch (bits) {
         case CQ_BITS_TERNARY:
-            e = launch_rotate<3>(x, sh, batch, codebook, xfrag, xscale, table, stream);
-            return e != cudaSuccess ? e : launch_gemv_bits<2>(packed, norms, sh, xf, xscale, table, batch, y, stream);
+            e = launch_rotate<2, 3>(x, sh, batch, codebook, xfrag, xscale, table, stream);
+            return e != cudaSuccess ? e : launch_gemv_bits<2>(packed, norms, sh, xf, xs, table, batch, y, stream);
         case 2:
-            e = launch_rotate<4>(x, sh, batch, codebook, xfrag, xscale, table, stream);
-            return e != cudaSuccess ? e : launch_gemv_bits<2>(packed, norms, sh, xf, xscale, table, batch, y, stream);
+            e = launch_rotate<2, 4>(x, sh, batch, codebook, xfrag, xscale, table, stream);
+            return e != cudaSuccess ? e : launch_gemv_bits<2>(packed, norms, sh, xf, xs, table, batch, y, stream);
         case 3:
-            e = launch_rotate<8>(x, sh, batch, codebook, xfrag, xscale, table, stream);
-            return e != cudaSuccess ? e : launch_gemv_bits<3>(packed, norms, sh, xf, xscale, table, batch, y, stream);
+            e = launch_rotate<3, 8>(x, sh, batch, codebook, xfrag, xscale, table, stream);
+            return e != cudaSuccess ? e : launch_gemv_bits<3>(packed, norms, sh, xf, xs, table, batch, y, stream);
         default:
-            e = launch_rotate<16>(x, sh, batch, codebook, xfrag, xscale, table, stream);
-            return e != cudaSuccess ? e : launch_gemv_bits<4>(packed, norms, sh, xf, xscale, table, batch, y, stream);
+            e = launch_rotate<4, 16>(x, sh, batch, codebook, xfrag, xscale, table, stream);
+            return e != cudaSuccess ? e : launch_gemv_bits<4>(packed, norms, sh, xf, xs, table, batch, y, stream);
     }
 }
 
