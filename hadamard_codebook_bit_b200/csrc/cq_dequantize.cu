@@ -88,6 +88,8 @@ __global__ void __launch_bounds__(kThreads)
                       long long cols, long long G, long long total,
                       const float* __restrict__ codebook, void* __restrict__ out) {
     __shared__ float cb_s[16];
+    pdl_trigger();
+    pdl_wait();
     if (threadIdx.x < 16) cb_s[threadIdx.x] = threadIdx.x < L ? codebook[threadIdx.x] : 0.0f;
     __syncthreads();
 
@@ -143,19 +145,15 @@ cudaError_t launch_mode(int mode, const uint8_t* packed, const uint16_t* norms, 
     const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(blocks_needed, max_blocks)));
     switch (mode) {
         case kFlat:
-            dequantize_kernel<B, L, kBF16, kFlat><<<grid, kThreads, 0, st>>>(
-                packed, norms, sh.cols, sh.groups_per_row, sh.total_groups, cb, out);
-            break;
+            return launch_pdl(dequantize_kernel<B, L, kBF16, kFlat>, dim3(grid), dim3(kThreads), 0, st,
+                              packed, norms, sh.cols, sh.groups_per_row, sh.total_groups, cb, out);
         case kVector:
-            dequantize_kernel<B, L, kBF16, kVector><<<grid, kThreads, 0, st>>>(
-                packed, norms, sh.cols, sh.groups_per_row, sh.total_groups, cb, out);
-            break;
+            return launch_pdl(dequantize_kernel<B, L, kBF16, kVector>, dim3(grid), dim3(kThreads), 0, st,
+                              packed, norms, sh.cols, sh.groups_per_row, sh.total_groups, cb, out);
         default:
-            dequantize_kernel<B, L, kBF16, kScalar><<<grid, kThreads, 0, st>>>(
-                packed, norms, sh.cols, sh.groups_per_row, sh.total_groups, cb, out);
-            break;
+            return launch_pdl(dequantize_kernel<B, L, kBF16, kScalar>, dim3(grid), dim3(kThreads), 0, st,
+                              packed, norms, sh.cols, sh.groups_per_row, sh.total_groups, cb, out);
     }
-    return cudaGetLastError();
 }
 
 template <int B, int L>

@@ -131,35 +131,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     uint8_t* stage_out = ring + kStagesDq * kStageBytes;  // 2 x OutTile (1024-aligned)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // codewords c_k 2^cs = hi_k + lo_k in fp16
-    float cmax = 0.0f;
-#pragma unroll
-    for (int k = 0; k < L; ++k) cmax = fmaxf(cmax, fabsf(__ldg(codebook + k)));
-    const int cs = (cmax > 0.0f) ? (13 - ilogbf(cmax)) : 0;
-    uint32_t hl[4], hh[4], ll[4], lh[4];  // bytes of hi / lo for codes 0..3
-    uint32_t th_lo = 0, th_hi = 0, tl_lo = 0, tl_hi = 0;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const float x = ldexpf(__ldg(codebook + (k < L ? k : L - 1)), cs);
-        const __half h = __float2half_rn(x);
-        const __half l = __float2half_rn(x - __half2float(h));
-        hl[k] = __half_as_ushort(h) & 0xffu;
-        hh[k] = __half_as_ushort(h) >> 8;
-        ll[k] = __half_as_ushort(l) & 0xffu;
-        lh[k] = __half_as_ushort(l) >> 8;
-        th_lo |= hl[k] << (8 * k);
-        th_hi |= hh[k] << (8 * k);
-        tl_lo |= ll[k] << (8 * k);
-        tl_hi |= lh[k] << (8 * k);
-    }
-    if (threadIdx.x < 16) {
-        const float x = ldexpf(__ldg(codebook + (threadIdx.x < L ? threadIdx.x : L - 1)), cs);
-        const __half h = __float2half_rn(x);
-        const __half l = __float2half_rn(x - __half2float(h));
-        tab_s[threadIdx.x] = static_cast<uint32_t>(__half_as_ushort(h)) |
-                             (static_cast<uint32_t>(__half_as_ushort(l)) << 16);
-    }
-    const float inv_scale = ldexpf(1.0f, -cs) * kInvSqrt128;
+    pdl_trigger();
+
 
     // B operand: row n, column k = H_int[n][e(k)] (fp16 +-1), K-major, 128-byte swizzle
     for (int item = threadIdx.x; item < kTile * 16; item += kDqThreads) {
@@ -194,6 +167,38 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = tmem_slot;
+    pdl_wait();  // on-chip set-up above; global memory only from here
+
+    // codewords c_k 2^cs = hi_k + lo_k in fp16
+    float cmax = 0.0f;
+#pragma unroll
+    for (int k = 0; k < L; ++k) cmax = fmaxf(cmax, fabsf(__ldg(codebook + k)));
+    const int cs = (cmax > 0.0f) ? (13 - ilogbf(cmax)) : 0;
+    uint32_t hl[4], hh[4], ll[4], lh[4];  // bytes of hi / lo for codes 0..3
+    uint32_t th_lo = 0, th_hi = 0, tl_lo = 0, tl_hi = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float x = ldexpf(__ldg(codebook + (k < L ? k : L - 1)), cs);
+        const __half h = __float2half_rn(x);
+        const __half l = __float2half_rn(x - __half2float(h));
+        hl[k] = __half_as_ushort(h) & 0xffu;
+        hh[k] = __half_as_ushort(h) >> 8;
+        ll[k] = __half_as_ushort(l) & 0xffu;
+        lh[k] = __half_as_ushort(l) >> 8;
+        th_lo |= hl[k] << (8 * k);
+        th_hi |= hh[k] << (8 * k);
+        tl_lo |= ll[k] << (8 * k);
+        tl_hi |= lh[k] << (8 * k);
+    }
+    if (threadIdx.x < 16) {
+        const float x = ldexpf(__ldg(codebook + (threadIdx.x < L ? threadIdx.x : L - 1)), cs);
+        const __half h = __float2half_rn(x);
+        const __half l = __float2half_rn(x - __half2float(h));
+        tab_s[threadIdx.x] = static_cast<uint32_t>(__half_as_ushort(h)) |
+                             (static_cast<uint32_t>(__half_as_ushort(l)) << 16);
+    }
+    const float inv_scale = ldexpf(1.0f, -cs) * kInvSqrt128;
+    __syncthreads();  // tab_s
 
     if (warp == 0) {
         // ---------------- bulk-copy producer ----------------
@@ -392,7 +397,11 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 template <int B, int L, bool kBF16>
 cudaError_t launch_dq(const uint8_t* packed, const uint16_t* norms, const DqShape& ds,
                       const float* cb, void* out, unsigned* status, cudaStream_t st) {
-    const int smem = kHBytes + kStagesDq * kTile * 16 * B + 2 * OutTile<kBF16>::kBytes + 1024;
+    // at least 120 KB so that two CTAs never share an SM: each takes all 512 TMEM columns, and
+    // with programmatic launch a CTA of the next kernel could otherwise wait inside
+    // tcgen05.alloc until the previous one frees them
+    const int smem = std::max(kHBytes + kStagesDq * kTile * 16 * B + 2 * OutTile<kBF16>::kBytes + 1024,
+                              120 * 1024);
     CUtensorMap omap;
     std::memset(&omap, 0, sizeof(omap));
     if (ds.flat) {
@@ -420,8 +429,8 @@ cudaError_t launch_dq(const uint8_t* packed, const uint16_t* norms, const DqShap
         configured |= bit;
     }
     const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(ds.tiles, sm_count())));
-    dequantize_tc_kernel<B, L, kBF16><<<grid, kDqThreads, smem, st>>>(packed, norms, ds, cb, out, status, omap);
-    return cudaGetLastError();
+    return launch_pdl(dequantize_tc_kernel<B, L, kBF16>, dim3(grid), dim3(kDqThreads), smem, st,
+                      packed, norms, ds, cb, out, status, omap);
 }
 
 template <int B, int L>

@@ -32,6 +32,17 @@ constexpr int kGroupsPerWarp = 8;
 constexpr float kInvSqrt128 = 0.088388347648318440550f;  // fp32(1/sqrt(128))
 
 // ---------------------------------------------------------------------------------------
+// programmatic dependent launch (see launch_pdl)
+// ---------------------------------------------------------------------------------------
+
+// Let the next kernel in the stream be scheduled; it still waits for this one to finish
+// before touching global memory.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Wait until the previous kernel in the stream has finished and its writes are visible.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------------------
 // memory helpers
 // ---------------------------------------------------------------------------------------
 

@@ -91,8 +91,8 @@ __global__ void __launch_bounds__(kRotThreads)
     rotate_x_kernel(const uint16_t* __restrict__ x, long long cols, long long G, int batch,
                     const float* __restrict__ codebook, __half* __restrict__ xfrag,
                     float* __restrict__ xscale, CodeTable* __restrict__ table) {
-    // the GEMV that follows may start its weight copies now (it waits before reading x~)
-    asm volatile("griddepcontrol.launch_dependents;");
+    pdl_trigger();  // the GEMV may be scheduled now; it waits for this kernel before any access
+    pdl_wait();
     const long long j = blockIdx.x;
     const int b = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -399,7 +399,8 @@ __global__ void __maxnreg__(96)
     // Nothing is read before the dependency wait: loads issued earlier by a programmatic
     // dependent (even of buffers written by kernels that ran before step 1) returned stale
     // data on this hardware.  The early launch still hides the launch latency.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    pdl_trigger();
+    pdl_wait();
     float inv_scale;
     load_tables<B>(table, st.tb, inv_scale);
 
@@ -461,26 +462,17 @@ cudaError_t launch_gemv_bits(const uint8_t* packed, const uint16_t* norms, const
                              int batch, float* y, cudaStream_t st) {
     const long long blocks = (sh.rows + kRowsPerBlock - 1) / kRowsPerBlock;
     const int split = gemv_split(blocks, sh.groups_per_row, gemv_regs<B>());
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(blocks));
-    cfg.blockDim = dim3(static_cast<unsigned>(32 * split));
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemv_split_kernel<B>, packed, norms, sh.rows,
-                              static_cast<int>(sh.groups_per_row), xfrag, xscale, table, batch, y);
+    return launch_pdl(gemv_split_kernel<B>, dim3(static_cast<unsigned>(blocks)), dim3(32 * split), 0, st,
+                      packed, norms, sh.rows, static_cast<int>(sh.groups_per_row), xfrag, xscale,
+                      table, batch, y);
 }
 
 template <int B, int L>
 cudaError_t launch_rotate(const uint16_t* x, const Shape& sh, int batch, const float* codebook,
                           __half* xfrag, float* xscale, CodeTable* table, cudaStream_t st) {
-    rotate_x_kernel<B, L><<<static_cast<unsigned>(sh.groups_per_row), kRotThreads, 0, st>>>(
-        x, sh.cols, sh.groups_per_row, batch, codebook, xfrag, xscale, table);
-    return cudaGetLastError();
+    return launch_pdl(rotate_x_kernel<B, L>, dim3(static_cast<unsigned>(sh.groups_per_row)),
+                      dim3(kRotThreads), 0, st, x, sh.cols, sh.groups_per_row, batch, codebook,
+                      xfrag, xscale, table);
 }
 
 }  // namespace

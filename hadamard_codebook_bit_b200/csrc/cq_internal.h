@@ -28,6 +28,28 @@ struct Shape {
     long long total_groups;    // rows * G
 };
 
+// Launch with programmatic stream serialization: the kernel may start while the previous
+// kernel in the stream is still running (after that kernel's griddepcontrol.launch_dependents).
+// Every kernel of this library therefore executes griddepcontrol.wait before its first global
+// memory access (read or write); only on-chip set-up (shared memory tables, barriers, tensor
+// memory) runs earlier.  Kernels that follow in the stream without this attribute still wait
+// for full completion.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Kernel launchers (one per file).  All return cudaSuccess or the launch error.
 // cuTensorMapEncodeTiled, looked up once through the runtime's driver entry point (nullptr
 // when unavailable).

@@ -89,6 +89,8 @@ __global__ void __launch_bounds__(kThreads)
     quantize_kernel(const void* __restrict__ w, long long cols, long long G, long long total,
                     const float* __restrict__ codebook, uint8_t* __restrict__ packed,
                     uint16_t* __restrict__ norms) {
+    pdl_trigger();
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int q = lane >> 2, s = lane & 3;
 
@@ -155,19 +157,15 @@ cudaError_t launch_mode(int mode, const void* w, const Shape& sh, const float* c
     const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(blocks_needed, max_blocks)));
     switch (mode) {
         case kFlat:
-            quantize_kernel<B, L, kBF16, kFlat><<<grid, kThreads, 0, st>>>(
-                w, sh.cols, sh.groups_per_row, sh.total_groups, cb, packed, norms);
-            break;
+            return launch_pdl(quantize_kernel<B, L, kBF16, kFlat>, dim3(grid), dim3(kThreads), 0, st,
+                              w, sh.cols, sh.groups_per_row, sh.total_groups, cb, packed, norms);
         case kVector:
-            quantize_kernel<B, L, kBF16, kVector><<<grid, kThreads, 0, st>>>(
-                w, sh.cols, sh.groups_per_row, sh.total_groups, cb, packed, norms);
-            break;
+            return launch_pdl(quantize_kernel<B, L, kBF16, kVector>, dim3(grid), dim3(kThreads), 0, st,
+                              w, sh.cols, sh.groups_per_row, sh.total_groups, cb, packed, norms);
         default:
-            quantize_kernel<B, L, kBF16, kScalar><<<grid, kThreads, 0, st>>>(
-                w, sh.cols, sh.groups_per_row, sh.total_groups, cb, packed, norms);
-            break;
+            return launch_pdl(quantize_kernel<B, L, kBF16, kScalar>, dim3(grid), dim3(kThreads), 0, st,
+                              w, sh.cols, sh.groups_per_row, sh.total_groups, cb, packed, norms);
     }
-    return cudaGetLastError();
 }
 
 template <int B, int L>

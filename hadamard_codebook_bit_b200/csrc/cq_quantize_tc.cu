@@ -124,6 +124,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint8_t* ring = smem + kTileBytes;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_trigger();
 
     // H_int (+1 = 0x3F80, -1 = 0xBF80 in bf16), row n = output element, column k = input element
     for (int item = threadIdx.x; item < kTile * 16; item += kTcThreads) {
@@ -157,6 +158,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = tmem_slot;
+    pdl_wait();  // on-chip set-up above; global memory only from here
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
@@ -307,8 +309,8 @@ cudaError_t launch_tc(const CUtensorMap& map, const TcShape& ts, const float* cb
         configured |= bit;
     }
     const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(ts.tiles, sm_count())));
-    quantize_tc_kernel<B, L><<<grid, kTcThreads, smem, st>>>(map, ts, cb, packed, norms, status);
-    return cudaGetLastError();
+    return launch_pdl(quantize_tc_kernel<B, L>, dim3(grid), dim3(kTcThreads), smem, st, map, ts, cb,
+                      packed, norms, status);
 }
 
 }  // namespace
