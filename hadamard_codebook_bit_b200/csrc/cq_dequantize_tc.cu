@@ -161,6 +161,14 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             mbar_init(&dfull_bar[a], 1);
         }
         fence_mbar_init();
+        // the first tiles' codes and norms of this CTA into L2 while the previous kernel finishes
+        long long t = blockIdx.x;
+        for (int i = 0; i < kStagesDq && t < sh.tiles; ++i, t += gridDim.x) {
+            const long long g0 = t * kTile;
+            const long long n = sh.total - g0 < kTile ? sh.total - g0 : kTile;
+            bulk_prefetch_l2(packed + g0 * (16 * B), static_cast<uint32_t>(n) * (16 * B));
+            if (n == kTile) bulk_prefetch_l2(norms + g0, kTile * 2);
+        }
     }
     if (warp == 1) tmem_alloc(&tmem_slot, kTmemColsDq);
     tc_fence_before();

@@ -152,6 +152,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         fence_mbar_init();
         prefetch_tensormap(&tmap);
+        // the first tiles of this CTA into L2 while the previous kernel finishes
+        long long t = blockIdx.x;
+        for (int i = 0; i < kStagesTc && t < sh.tiles; ++i, t += gridDim.x) {
+            const int rb = static_cast<int>(t % sh.tiles_r), j = static_cast<int>(t / sh.tiles_r);
+            tma_prefetch_2d(&tmap, kTile * j, kTile * rb);
+            tma_prefetch_2d(&tmap, kTile * j + 64, kTile * rb);
+        }
     }
     if (warp == 1) tmem_alloc(&tmem_slot, kTmemCols);
     tc_fence_before();
