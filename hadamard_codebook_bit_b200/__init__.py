@@ -29,7 +29,8 @@ _STATUS = {0: "CQ_OK", 1: "CQ_ERR_INVALID_ARG", 2: "CQ_ERR_UNSUPPORTED", 3: "CQ_
 # Every symbol include/cq.h declares (checked by the CPU test suite).
 EXPORTS = ("cq_status_string", "cq_version", "cq_device_status", "cq_codebook", "cq_packed_bytes",
            "cq_norm_bytes", "cq_quantize", "cq_dequantize", "cq_dequant_gemv",
-           "cq_gemv_workspace_bytes", "cq_dequant_gemv_static")
+           "cq_gemv_workspace_bytes", "cq_dequant_gemv_static", "cq_quantize_batch",
+           "cq_dequantize_batch")
 
 
 class CQError(RuntimeError):
@@ -65,6 +66,8 @@ def lib() -> ctypes.CDLL:
         L.cq_gemv_workspace_bytes.argtypes = [ll, i]
         L.cq_gemv_workspace_bytes.restype = sz
         L.cq_dequant_gemv_static.argtypes = [P, P, ll, ll, i, i, P, P, i, P, P]
+        L.cq_quantize_batch.argtypes = [P, i, i, i, i, P, P]
+        L.cq_dequantize_batch.argtypes = [P, i, i, i, P, i, P]
         _lib = L
     return _lib
 
@@ -167,6 +170,78 @@ def quantize(w, bits: int, group_size: int = GROUP_SIZE, codebook=None, out=None
                                  _cb_ptr(codebook, w.device), _dev_ptr(packed, "packed"),
                                  _dev_ptr(norms, "norms"), _stream(w.device)), "cq_quantize")
     return packed, norms
+
+
+class _QuantizeJob(ctypes.Structure):  # cq_quantize_job
+    _fields_ = [("w", ctypes.c_void_p), ("rows", ctypes.c_longlong), ("cols", ctypes.c_longlong),
+                ("packed_out", ctypes.c_void_p), ("norms_out", ctypes.c_void_p)]
+
+
+class _DequantizeJob(ctypes.Structure):  # cq_dequantize_job
+    _fields_ = [("packed", ctypes.c_void_p), ("norms", ctypes.c_void_p), ("rows", ctypes.c_longlong),
+                ("cols", ctypes.c_longlong), ("out", ctypes.c_void_p)]
+
+
+def quantize_batch(ws, bits: int, group_size: int = GROUP_SIZE, codebook=None, outs=None):
+    """cq_quantize_batch on a list of 2-D CUDA tensors of one dtype (bf16 or fp32) on one
+    device -> list of (packed, norms).  `outs`, if given, is a list of (packed, norms)."""
+    torch = _torch()
+    if not ws:
+        return []
+    dev, dtype = ws[0].device, ws[0].dtype
+    if dtype == torch.bfloat16:
+        dt = CQ_BF16
+    elif dtype == torch.float32:
+        dt = CQ_F32
+    else:
+        raise ValueError("tensors must be bfloat16 or float32")
+    jobs = (_QuantizeJob * len(ws))()
+    res = []
+    for k, w in enumerate(ws):
+        if w.dim() != 2 or w.dtype != dtype or w.device != dev:
+            raise ValueError("tensors must be 2-D, of one dtype, on one device")
+        rows, cols = w.shape
+        packed, norms = outs[k] if outs is not None else empty_packed(rows, cols, bits, dev, group_size)
+        jobs[k] = _QuantizeJob(_dev_ptr(w, "w"), rows, cols, _dev_ptr(packed, "packed"),
+                               _dev_ptr(norms, "norms"))
+        res.append((packed, norms))
+    with torch.cuda.device(dev):
+        _check(lib().cq_quantize_batch(ctypes.cast(jobs, ctypes.c_void_p), len(ws), dt, bits, group_size,
+                                       _cb_ptr(codebook, dev), _stream(dev)), "cq_quantize_batch")
+    return res
+
+
+def dequantize_batch(items, bits: int, group_size: int = GROUP_SIZE, codebook=None,
+                     out_dtype=None, outs=None):
+    """cq_dequantize_batch on a list of (packed, norms, rows, cols) on one device -> list of
+    W_hat tensors (bfloat16 by default, or float32; `outs` gives them)."""
+    torch = _torch()
+    if not items:
+        return []
+    dev = items[0][0].device
+    if outs is None:
+        out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+        outs = [torch.empty((r, c), dtype=out_dtype, device=dev) for _, _, r, c in items]
+    dtype = outs[0].dtype
+    if dtype == torch.bfloat16:
+        dt = CQ_BF16
+    elif dtype == torch.float32:
+        dt = CQ_F32
+    else:
+        raise ValueError("out dtype must be bfloat16 or float32")
+    jobs = (_DequantizeJob * len(items))()
+    for k, ((packed, norms, rows, cols), out) in enumerate(zip(items, outs)):
+        if norms.dtype != torch.float16:
+            raise ValueError("norms must be float16")
+        if out.dtype != dtype or packed.device != dev or out.device != dev:
+            raise ValueError("outputs must share one dtype and device")
+        jobs[k] = _DequantizeJob(_dev_ptr(packed, "packed"), _dev_ptr(norms, "norms"), rows, cols,
+                                 _dev_ptr(out, "out"))
+    with torch.cuda.device(dev):
+        _check(lib().cq_dequantize_batch(ctypes.cast(jobs, ctypes.c_void_p), len(items), bits,
+                                         group_size, _cb_ptr(codebook, dev), dt, _stream(dev)),
+               "cq_dequantize_batch")
+    return outs
 
 
 def dequantize(packed, norms, rows: int, cols: int, bits: int, group_size: int = GROUP_SIZE,

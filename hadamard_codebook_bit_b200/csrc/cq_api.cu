@@ -6,6 +6,8 @@
 #include <cstdlib>
 #include <mutex>
 
+#include <vector>
+
 #include "cq_internal.h"
 
 namespace cq {
@@ -226,6 +228,87 @@ int cq_dequantize(const unsigned char* packed, const unsigned short* norms, long
                                                 cb, out, out_dtype,
                                                 static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
+}
+
+int cq_quantize_batch(const cq_quantize_job* jobs, int count, int w_dtype, int bits,
+                      int group_size, const float* codebook, void* stream) {
+    if (count < 0 || (count > 0 && !jobs)) return CQ_ERR_INVALID_ARG;
+    if (w_dtype != CQ_F32 && w_dtype != CQ_BF16) return CQ_ERR_INVALID_ARG;
+    for (int i = 0; i < count; ++i) {
+        const cq_quantize_job& j = jobs[i];
+        const int rc = cq::check_common(j.rows, j.cols, bits, group_size);
+        if (rc != CQ_OK) return rc;
+        if (j.rows == 0 || j.cols == 0) continue;
+        if (!j.w || !j.packed_out || !j.norms_out) return CQ_ERR_INVALID_ARG;
+        if (!cq::aligned16(j.w) || !cq::aligned16(j.packed_out) || !cq::aligned16(j.norms_out))
+            return CQ_ERR_ALIGNMENT;
+    }
+    bool any = false;
+    for (int i = 0; i < count; ++i) any = any || (jobs[i].rows > 0 && jobs[i].cols > 0);
+    if (!any) return CQ_OK;  // nothing to quantise
+    const float* cb = nullptr;
+    int rc = cq::resolve_codebook(bits, codebook, &cb);
+    if (rc != CQ_OK) return rc;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    std::vector<cq::QuantizeItem> tc;
+    unsigned* status = cq::device_status_ptr();
+    for (int i = 0; i < count; ++i) {
+        const cq_quantize_job& j = jobs[i];
+        if (j.rows == 0 || j.cols == 0) continue;
+        const cq::Shape sh = cq::make_shape(j.rows, j.cols);
+        if (status && cq::tcgen05_enabled() && cq::quantize_tc_supported(w_dtype, sh)) {
+            tc.push_back({j.w, sh, j.packed_out, j.norms_out});
+        } else {
+            const cudaError_t e = cq::launch_quantize(j.w, w_dtype, sh, bits, cb, j.packed_out, j.norms_out, st);
+            if (e != cudaSuccess) return CQ_ERR_CUDA;
+        }
+    }
+    if (!tc.empty()) {
+        const cudaError_t e = cq::launch_quantize_tc_batch(tc.data(), static_cast<int>(tc.size()), bits, cb, status, st);
+        if (e != cudaSuccess) return CQ_ERR_CUDA;
+    }
+    return CQ_OK;
+}
+
+int cq_dequantize_batch(const cq_dequantize_job* jobs, int count, int bits, int group_size,
+                        const float* codebook, int out_dtype, void* stream) {
+    if (count < 0 || (count > 0 && !jobs)) return CQ_ERR_INVALID_ARG;
+    if (out_dtype != CQ_F32 && out_dtype != CQ_BF16) return CQ_ERR_INVALID_ARG;
+    for (int i = 0; i < count; ++i) {
+        const cq_dequantize_job& j = jobs[i];
+        const int rc = cq::check_common(j.rows, j.cols, bits, group_size);
+        if (rc != CQ_OK) return rc;
+        if (j.rows == 0 || j.cols == 0) continue;
+        if (!j.packed || !j.norms || !j.out) return CQ_ERR_INVALID_ARG;
+        if (!cq::aligned16(j.packed) || !cq::aligned16(j.norms) || !cq::aligned16(j.out))
+            return CQ_ERR_ALIGNMENT;
+    }
+    bool any = false;
+    for (int i = 0; i < count; ++i) any = any || (jobs[i].rows > 0 && jobs[i].cols > 0);
+    if (!any) return CQ_OK;  // nothing to write
+    const float* cb = nullptr;
+    int rc = cq::resolve_codebook(bits, codebook, &cb);
+    if (rc != CQ_OK) return rc;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    std::vector<cq::DequantizeItem> tc;
+    unsigned* status = cq::device_status_ptr();
+    for (int i = 0; i < count; ++i) {
+        const cq_dequantize_job& j = jobs[i];
+        if (j.rows == 0 || j.cols == 0) continue;
+        const cq::Shape sh = cq::make_shape(j.rows, j.cols);
+        if (status && cq::tcgen05_enabled() && cq::dequantize_tc_supported(out_dtype, sh)) {
+            tc.push_back({j.packed, j.norms, sh, j.out});
+        } else {
+            const cudaError_t e = cq::launch_dequantize(j.packed, j.norms, sh, bits, cb, j.out, out_dtype, st);
+            if (e != cudaSuccess) return CQ_ERR_CUDA;
+        }
+    }
+    if (!tc.empty()) {
+        const cudaError_t e = cq::launch_dequantize_tc_batch(tc.data(), static_cast<int>(tc.size()), bits, cb,
+                                                             out_dtype, status, st);
+        if (e != cudaSuccess) return CQ_ERR_CUDA;
+    }
+    return CQ_OK;
 }
 
 size_t cq_gemv_workspace_bytes(long long cols, int batch) {

@@ -25,6 +25,7 @@
 // shift + mask, and row n of the shared-memory B holds H_int[n][e(k)].
 #include <algorithm>
 #include <cstring>
+#include <mutex>
 
 #include "cq_device.cuh"
 #include "cq_internal.h"
@@ -52,6 +53,34 @@ struct DqShape {
     long long tiles;   // ceil(total / 128)
     int flat;          // cols % 128 == 0: group g's output starts at element 128 g
 };
+
+// The tensors of one launch.  Job k owns the global tiles [tile0[k], tile0[k + 1]); omap[k]
+// is the output tensor map of a flat job.
+template <int NJ>
+struct DqJobs {
+    CUtensorMap omap[NJ];  // 64-byte aligned, first
+    DqShape sh[NJ];
+    const uint8_t* packed[NJ];
+    const uint16_t* norms[NJ];
+    void* out[NJ];
+    long long tile0[NJ + 1];
+    int n;
+};
+
+template <int NJ>
+__device__ __forceinline__ int job_of(const DqJobs<NJ>& jb, long long t) {
+    if constexpr (NJ == 1) {
+        return 0;
+    } else {
+        int lo = 0, hi = jb.n - 1;  // largest k with tile0[k] <= t
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (jb.tile0[mid] <= t) lo = mid;
+            else hi = mid - 1;
+        }
+        return lo;
+    }
+}
 
 // Element of the group held by MMA column k.
 template <int B>
@@ -113,11 +142,10 @@ struct OutTile {
     }
 };
 
-template <int B, int L, bool kBF16>
+template <int B, int L, bool kBF16, int NJ>
 __global__ void __launch_bounds__(kDqThreads, 1)
-    dequantize_tc_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ norms,
-                         DqShape sh, const float* __restrict__ codebook, void* __restrict__ out,
-                         unsigned* __restrict__ status, const __grid_constant__ CUtensorMap omap) {
+    dequantize_tc_kernel(const __grid_constant__ DqJobs<NJ> jobs, const float* __restrict__ codebook,
+                         unsigned* __restrict__ status) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full_bar[kStagesDq], empty_bar[kStagesDq];
     __shared__ __align__(8) uint64_t afull_bar[2], dfull_bar[2];
@@ -130,6 +158,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     uint8_t* ring = smem + kHBytes;
     uint8_t* stage_out = ring + kStagesDq * kStageBytes;  // 2 x OutTile (1024-aligned)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long ntiles = jobs.tile0[jobs.n];
 
     pdl_trigger();
 
@@ -163,11 +192,13 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         fence_mbar_init();
         // the first tiles' codes and norms of this CTA into L2 while the previous kernel finishes
         long long t = blockIdx.x;
-        for (int i = 0; i < kStagesDq && t < sh.tiles; ++i, t += gridDim.x) {
-            const long long g0 = t * kTile;
+        for (int i = 0; i < kStagesDq && t < ntiles; ++i, t += gridDim.x) {
+            const int k = job_of(jobs, t);
+            const DqShape& sh = jobs.sh[k];
+            const long long g0 = (t - jobs.tile0[k]) * kTile;
             const long long n = sh.total - g0 < kTile ? sh.total - g0 : kTile;
-            bulk_prefetch_l2(packed + g0 * (16 * B), static_cast<uint32_t>(n) * (16 * B));
-            if (n == kTile) bulk_prefetch_l2(norms + g0, kTile * 2);
+            bulk_prefetch_l2(jobs.packed[k] + g0 * (16 * B), static_cast<uint32_t>(n) * (16 * B));
+            if (n == kTile) bulk_prefetch_l2(jobs.norms[k] + g0, kTile * 2);
         }
     }
     if (warp == 1) tmem_alloc(&tmem_slot, kTmemColsDq);
@@ -212,14 +243,16 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         // ---------------- bulk-copy producer ----------------
         if (lane == 0) {
             int i = 0;
-            for (long long t = blockIdx.x; t < sh.tiles; t += gridDim.x, ++i) {
+            for (long long t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
                 const int st = i % kStagesDq;
                 if (!mbar_wait(&empty_bar[st], ((i / kStagesDq) & 1) ^ 1, status)) break;
-                const long long g0 = t * kTile;
+                const int k = job_of(jobs, t);
+                const DqShape& sh = jobs.sh[k];
+                const long long g0 = (t - jobs.tile0[k]) * kTile;
                 const long long n = sh.total - g0 < kTile ? sh.total - g0 : kTile;
                 const uint32_t bytes = static_cast<uint32_t>(n) * (16 * B);
                 mbar_arrive_expect_tx(&full_bar[st], bytes);
-                bulk_load(ring + st * kStageBytes, packed + g0 * (16 * B), bytes, &full_bar[st]);
+                bulk_load(ring + st * kStageBytes, jobs.packed[k] + g0 * (16 * B), bytes, &full_bar[st]);
             }
             for (int k = 0; k < kStagesDq && k < i; ++k) {
                 const int ii = i - 1 - k;
@@ -230,7 +263,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
             int i = 0;
-            for (long long t = blockIdx.x; t < sh.tiles; t += gridDim.x, ++i) {
+            for (long long t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
                 const int e = i & 1;
                 if (!mbar_wait(&afull_bar[e], (i >> 1) & 1, status)) break;
                 tc_fence_after();
@@ -257,12 +290,15 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
         const uint32_t a_hi = tbase + lane_off + e * kSlotCols, a_lo = a_hi + 64, d = a_hi + 128;
         int i = e;
-        for (long long t = blockIdx.x + static_cast<long long>(e) * gridDim.x; t < sh.tiles;
+        for (long long t = blockIdx.x + static_cast<long long>(e) * gridDim.x; t < ntiles;
              t += 2LL * gridDim.x, i += 2) {
+            const int k = job_of(jobs, t);
+            const DqShape& sh = jobs.sh[k];
+            const long long tl = t - jobs.tile0[k];
             const int st = i % kStagesDq;
             // the group's four warps decide together whether to go on
             if (!named_barrier_and(1 + e, 128, mbar_wait(&full_bar[st], (i / kStagesDq) & 1, status))) break;
-            const long long gid = t * kTile + m;
+            const long long gid = tl * kTile + m;
             const bool valid = gid < sh.total;
             uint32_t wd[4 * B];
             {
@@ -276,7 +312,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                     wd[4 * v + 3] = u.w;
                 }
             }
-            const float nrm = valid ? __half2float(__ushort_as_half(__ldg(norms + gid))) : 0.0f;
+            const float nrm = valid ? __half2float(__ushort_as_half(__ldg(jobs.norms[k] + gid))) : 0.0f;
 
             // A planes: 64 columns each, written 32 at a time
 #pragma unroll
@@ -369,7 +405,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                 if (leader) {
 #pragma unroll
                     for (int b = 0; b < OutTile<kBF16>::kBoxes; ++b)
-                        tma_store_2d(&omap, b * OutTile<kBF16>::kPerBox, static_cast<int>(t * kTile),
+                        tma_store_2d(&jobs.omap[k], b * OutTile<kBF16>::kPerBox, static_cast<int>(tl * kTile),
                                      so + b * OutTile<kBF16>::kBoxBytes);
                     bulk_commit();
                 }
@@ -386,12 +422,12 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                     for (int q = 0; q < 32 / kPer; ++q) {
                         const int off = q * kPer;
                         if (j * kTile + 32 * c + off < sh.cols)
-                            store_chunk<kBF16>(out, base + 32 * c + off, v, off, scale);
+                            store_chunk<kBF16>(jobs.out[k], base + 32 * c + off, v, off, scale);
                     }
                 }
             }
         }
-        if (sh.flat && (warp == 2 + 4 * e) && lane == 0) bulk_wait0();  // stores done before exit
+        if ((warp == 2 + 4 * e) && lane == 0) bulk_wait0();  // tensor-map stores done before exit
     }
 
     tc_fence_before();
@@ -402,52 +438,81 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     }
 }
 
-template <int B, int L, bool kBF16>
-cudaError_t launch_dq(const uint8_t* packed, const uint16_t* norms, const DqShape& ds,
-                      const float* cb, void* out, unsigned* status, cudaStream_t st) {
+template <int B, int L, bool kBF16, int NJ>
+cudaError_t launch_dq(const DqJobs<NJ>& jobs, const float* cb, unsigned* status, cudaStream_t st) {
     // at least 120 KB so that two CTAs never share an SM: each takes all 512 TMEM columns, and
     // with programmatic launch a CTA of the next kernel could otherwise wait inside
     // tcgen05.alloc until the previous one frees them
     const int smem = std::max(kHBytes + kStagesDq * kTile * 16 * B + 2 * OutTile<kBF16>::kBytes + 1024,
                               120 * 1024);
-    CUtensorMap omap;
-    std::memset(&omap, 0, sizeof(omap));
-    if (ds.flat) {
-        // the output viewed as [groups x 128] values, boxes of 128 bytes x 128 rows
-        const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(kTile), static_cast<cuuint64_t>(ds.total)};
-        const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(kTile) * (kBF16 ? 2 : 4)};
-        const cuuint32_t box[2] = {static_cast<cuuint32_t>(OutTile<kBF16>::kPerBox), kTile};
-        const cuuint32_t estride[2] = {1, 1};
-        EncodeTiledFn enc = tensor_map_encoder();
-        if (enc == nullptr) return cudaErrorNotSupported;
-        const CUresult r = enc(&omap, kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                               2, out, gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    }
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    static unsigned long long configured = 0;
+    static unsigned long long configured = 0;  // one bit per device
     const unsigned long long bit = 1ull << (dev & 63);
     if (!(configured & bit)) {
-        e = cudaFuncSetAttribute(dequantize_tc_kernel<B, L, kBF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        e = cudaFuncSetAttribute(dequantize_tc_kernel<B, L, kBF16, NJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         configured |= bit;
     }
-    const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(ds.tiles, sm_count())));
-    return launch_pdl(dequantize_tc_kernel<B, L, kBF16>, dim3(grid), dim3(kDqThreads), smem, st,
-                      packed, norms, ds, cb, out, status, omap);
+    const long long ntiles = jobs.tile0[jobs.n];
+    const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(ntiles, sm_count())));
+    return launch_pdl(dequantize_tc_kernel<B, L, kBF16, NJ>, dim3(grid), dim3(kDqThreads), smem, st,
+                      jobs, cb, status);
 }
 
-template <int B, int L>
-cudaError_t launch_dq_dtype(int out_dtype, const uint8_t* packed, const uint16_t* norms,
-                            const DqShape& ds, const float* cb, void* out, unsigned* status,
-                            cudaStream_t st) {
-    if (out_dtype == CQ_BF16) return launch_dq<B, L, true>(packed, norms, ds, cb, out, status, st);
-    return launch_dq<B, L, false>(packed, norms, ds, cb, out, status, st);
+// Shape, outputs and (flat shapes) the output tensor map of one tensor as job k of `jobs`.
+template <int NJ>
+bool add_job(DqJobs<NJ>& jobs, int k, const uint8_t* packed, const uint16_t* norms,
+             const Shape& sh, void* out, bool bf16) {
+    DqShape ds;
+    ds.total = sh.total_groups;
+    ds.cols = sh.cols;
+    ds.G = sh.groups_per_row;
+    ds.tiles = (sh.total_groups + kTile - 1) / kTile;
+    ds.flat = sh.cols % kTile == 0;
+    std::memset(&jobs.omap[k], 0, sizeof(CUtensorMap));
+    if (ds.flat) {
+        // the output viewed as [groups x 128] values, boxes of 128 bytes x 128 rows
+        const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(kTile), static_cast<cuuint64_t>(ds.total)};
+        const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(kTile) * (bf16 ? 2 : 4)};
+        const cuuint32_t box[2] = {static_cast<cuuint32_t>(bf16 ? OutTile<true>::kPerBox : OutTile<false>::kPerBox), kTile};
+        const cuuint32_t estride[2] = {1, 1};
+        EncodeTiledFn enc = tensor_map_encoder();
+        if (enc == nullptr) return false;
+        const CUresult r = enc(&jobs.omap[k], bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                               2, out, gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return false;
+    }
+    jobs.sh[k] = ds;
+    jobs.packed[k] = packed;
+    jobs.norms[k] = norms;
+    jobs.out[k] = out;
+    jobs.tile0[k + 1] = jobs.tile0[k] + ds.tiles;
+    return true;
 }
+
+template <int NJ>
+cudaError_t launch_bits(int bits, int out_dtype, const DqJobs<NJ>& jobs, const float* cb,
+                        unsigned* status, cudaStream_t st) {
+    const bool bf = out_dtype == CQ_BF16;
+    switch (bits) {
+        case CQ_BITS_TERNARY:
+            return bf ? launch_dq<2, 3, true, NJ>(jobs, cb, status, st) : launch_dq<2, 3, false, NJ>(jobs, cb, status, st);
+        case 2:
+            return bf ? launch_dq<2, 4, true, NJ>(jobs, cb, status, st) : launch_dq<2, 4, false, NJ>(jobs, cb, status, st);
+        case 3:
+            return bf ? launch_dq<3, 8, true, NJ>(jobs, cb, status, st) : launch_dq<3, 8, false, NJ>(jobs, cb, status, st);
+        default:
+            return bf ? launch_dq<4, 16, true, NJ>(jobs, cb, status, st) : launch_dq<4, 16, false, NJ>(jobs, cb, status, st);
+    }
+}
+
+// Jobs per batched launch: the job list travels in the kernel parameters (at most 32 KB).
+constexpr int kBatchJobs = 128;
+static_assert(sizeof(DqJobs<kBatchJobs>) < 32000, "kernel parameter space");
 
 }  // namespace
 
@@ -460,18 +525,32 @@ bool dequantize_tc_supported(int out_dtype, const Shape& sh) {
 cudaError_t launch_dequantize_tc(const uint8_t* packed, const uint16_t* norms, const Shape& sh,
                                  int bits, const float* codebook, void* out, int out_dtype,
                                  unsigned* status, cudaStream_t stream) {
-    DqShape ds;
-    ds.total = sh.total_groups;
-    ds.cols = sh.cols;
-    ds.G = sh.groups_per_row;
-    ds.tiles = (sh.total_groups + kTile - 1) / kTile;
-    ds.flat = sh.cols % kTile == 0;
-    switch (bits) {
-        case CQ_BITS_TERNARY: return launch_dq_dtype<2, 3>(out_dtype, packed, norms, ds, codebook, out, status, stream);
-        case 2: return launch_dq_dtype<2, 4>(out_dtype, packed, norms, ds, codebook, out, status, stream);
-        case 3: return launch_dq_dtype<3, 8>(out_dtype, packed, norms, ds, codebook, out, status, stream);
-        default: return launch_dq_dtype<4, 16>(out_dtype, packed, norms, ds, codebook, out, status, stream);
+    DqJobs<1> jobs;
+    jobs.n = 1;
+    jobs.tile0[0] = 0;
+    if (!add_job(jobs, 0, packed, norms, sh, out, out_dtype == CQ_BF16)) return cudaErrorInvalidValue;
+    return launch_bits(bits, out_dtype, jobs, codebook, status, stream);
+}
+
+cudaError_t launch_dequantize_tc_batch(const DequantizeItem* items, int count, int bits,
+                                       const float* codebook, int out_dtype, unsigned* status,
+                                       cudaStream_t stream) {
+    static DqJobs<kBatchJobs> jobs;  // host staging (large); calls are serialised below
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i0 = 0; i0 < count; i0 += kBatchJobs) {
+        const int n = std::min(kBatchJobs, count - i0);
+        jobs.n = n;
+        jobs.tile0[0] = 0;
+        for (int k = 0; k < n; ++k) {
+            const DequantizeItem& it = items[i0 + k];
+            if (!add_job(jobs, k, it.packed, it.norms, it.sh, it.out, out_dtype == CQ_BF16))
+                return cudaErrorInvalidValue;
+        }
+        const cudaError_t e = launch_bits(bits, out_dtype, jobs, codebook, status, stream);
+        if (e != cudaSuccess) return e;
     }
+    return cudaSuccess;
 }
 
 }  // namespace cq

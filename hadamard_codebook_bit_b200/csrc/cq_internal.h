@@ -67,17 +67,38 @@ unsigned* device_status_ptr();
 // (environment variable CQ_DISABLE_TCGEN05 unset or "0").
 bool tcgen05_enabled();
 
+// One tensor of a batched call.
+struct QuantizeItem {
+    const void* w;
+    Shape sh;
+    uint8_t* packed;
+    uint16_t* norms;
+};
+struct DequantizeItem {
+    const uint8_t* packed;
+    const uint16_t* norms;
+    Shape sh;
+    void* out;
+};
+
 // Tensor-core quantiser (cq_quantize_tc.cu): bf16 input, cols % 8 == 0.
 bool quantize_tc_supported(int w_dtype, const Shape& s);
 cudaError_t launch_quantize_tc(const void* w, const Shape& s, int bits, const float* codebook,
                                uint8_t* packed, uint16_t* norms, unsigned* status,
                                cudaStream_t stream);
+// Several tensors (each quantize_tc_supported, none empty) in as few launches as possible.
+cudaError_t launch_quantize_tc_batch(const QuantizeItem* items, int count, int bits,
+                                     const float* codebook, unsigned* status, cudaStream_t stream);
 
 // Tensor-core dequantiser (cq_dequantize_tc.cu): rows of the output start on 16 bytes.
 bool dequantize_tc_supported(int out_dtype, const Shape& s);
 cudaError_t launch_dequantize_tc(const uint8_t* packed, const uint16_t* norms, const Shape& s,
                                  int bits, const float* codebook, void* out, int out_dtype,
                                  unsigned* status, cudaStream_t stream);
+// Several tensors (each dequantize_tc_supported, none empty) in as few launches as possible.
+cudaError_t launch_dequantize_tc_batch(const DequantizeItem* items, int count, int bits,
+                                       const float* codebook, int out_dtype, unsigned* status,
+                                       cudaStream_t stream);
 
 cudaError_t launch_quantize(const void* w, int w_dtype, const Shape& s, int bits,
                             const float* codebook, uint8_t* packed, uint16_t* norms,

@@ -8,16 +8,18 @@
 // rotation ("rot @ H", page "How CQ2-bit Quantization Contributes to Needle 2's Small
 // Footprint", "Hadamard Rotation").
 //
-// Persistent kernel, one 320-thread CTA per SM:
+// Persistent kernel, one 576-thread CTA per SM:
 //   warp 0      TMA producer: 128 x 128 bf16 tiles (two 64-column boxes, 128-byte swizzle)
 //               into a 4-stage shared-memory ring;
-//   warp 1      owns 256 TMEM columns; one lane issues 8 tcgen05.mma (M=128, N=128, K=16)
-//               per tile into one of two TMEM accumulators, then commits to the stage's
+//   warp 1      owns 512 TMEM columns; one lane issues 8 tcgen05.mma (M=128, N=128, K=16)
+//               per tile into one of four TMEM accumulators, then commits to the stage's
 //               "empty" barrier and the accumulator's "full" barrier;
-//   warps 2-9   two epilogue groups of four warps (one per TMEM lane quadrant) take
-//               alternating tiles: each thread reads its group's 128 rotated values from
-//               TMEM, forms the norm, the thresholds m_k * ||r||, the indices, and stores
-//               the packed block and the fp16 norm.
+//   warps 2-17  four epilogue groups of four warps (one per TMEM lane quadrant) take tiles in
+//               turn: each thread reads its group's 128 rotated values from TMEM, forms the
+//               norm, the thresholds m_k * ||r||, the indices, and stores the packed block and
+//               the fp16 norm.
+// One launch may cover several tensors (a job list in the kernel parameters): the tiles of
+// all jobs form one index space that the CTAs stride through.
 // H_int lives in shared memory in the same swizzled K-major layout (built once per CTA).
 //
 // Tile -> groups: the tensor map views W as [R_eff rows x C_eff cols]; tile (rb, j) covers
@@ -26,6 +28,7 @@
 // cols % 128 == 0 the whole matrix is viewed as [groups x 128] (G_eff = 1), so one tile is
 // 128 consecutive groups and the packed output of a tile is one contiguous block.
 #include <algorithm>
+#include <mutex>
 
 #include "cq_device.cuh"
 #include "cq_internal.h"
@@ -49,6 +52,33 @@ constexpr uint32_t kIdesc = idesc_bf16_f32(kTile, kTile);
 struct TcShape {
     long long r_eff, g_eff, tiles_r, tiles;
 };
+
+// The tensors of one launch.  Job k owns the global tiles [tile0[k], tile0[k + 1]).
+template <int NJ>
+struct TcJobs {
+    CUtensorMap map[NJ];  // 64-byte aligned, first
+    TcShape sh[NJ];
+    uint8_t* packed[NJ];
+    uint16_t* norms[NJ];
+    long long tile0[NJ + 1];
+    int n;
+};
+
+// Job of global tile t (largest k with tile0[k] <= t).
+template <int NJ>
+__device__ __forceinline__ int job_of(const TcJobs<NJ>& jb, long long t) {
+    if constexpr (NJ == 1) {
+        return 0;
+    } else {
+        int lo = 0, hi = jb.n - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (jb.tile0[mid] <= t) lo = mid;
+            else hi = mid - 1;
+        }
+        return lo;
+    }
+}
 
 // Byte offset of element (row, k) of a 128 x 128 bf16 K-major tile stored as two 64-column
 // halves, each with the 128-byte swizzle (16-byte chunk index XOR row % 8).
@@ -108,11 +138,10 @@ __device__ __forceinline__ uint32_t pack2_signbits(const float (&v)[32], const f
     return w;
 }
 
-template <int B, int L>
+template <int B, int L, int NJ>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    quantize_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcShape sh,
-                       const float* __restrict__ codebook, uint8_t* __restrict__ packed,
-                       uint16_t* __restrict__ norms, unsigned* __restrict__ status) {
+    quantize_tc_kernel(const __grid_constant__ TcJobs<NJ> jobs, const float* __restrict__ codebook,
+                       unsigned* __restrict__ status) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full_bar[kStagesTc], empty_bar[kStagesTc];
     __shared__ __align__(8) uint64_t tfull_bar[kEpiGroups], tempty_bar[kEpiGroups];
@@ -124,6 +153,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint8_t* ring = smem + kTileBytes;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long ntiles = jobs.tile0[jobs.n];
     pdl_trigger();
 
     // H_int (+1 = 0x3F80, -1 = 0xBF80 in bf16), row n = output element, column k = input element
@@ -151,13 +181,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(&tempty_bar[a], 4);
         }
         fence_mbar_init();
-        prefetch_tensormap(&tmap);
         // the first tiles of this CTA into L2 while the previous kernel finishes
         long long t = blockIdx.x;
-        for (int i = 0; i < kStagesTc && t < sh.tiles; ++i, t += gridDim.x) {
-            const int rb = static_cast<int>(t % sh.tiles_r), j = static_cast<int>(t / sh.tiles_r);
-            tma_prefetch_2d(&tmap, kTile * j, kTile * rb);
-            tma_prefetch_2d(&tmap, kTile * j + 64, kTile * rb);
+        for (int i = 0; i < kStagesTc && t < ntiles; ++i, t += gridDim.x) {
+            const int k = job_of(jobs, t);
+            const TcShape& sh = jobs.sh[k];
+            const long long tl = t - jobs.tile0[k];
+            const int rb = static_cast<int>(tl % sh.tiles_r), j = static_cast<int>(tl / sh.tiles_r);
+            tma_prefetch_2d(&jobs.map[k], kTile * j, kTile * rb);
+            tma_prefetch_2d(&jobs.map[k], kTile * j + 64, kTile * rb);
         }
     }
     if (warp == 1) tmem_alloc(&tmem_slot, kTmemCols);
@@ -171,16 +203,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // ---------------- TMA producer ----------------
         if (lane == 0) {
             int i = 0;
-            for (long long t = blockIdx.x; t < sh.tiles; t += gridDim.x, ++i) {
+            for (long long t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
                 const int st = i % kStagesTc;
                 const uint32_t ph = (i / kStagesTc) & 1;
                 if (!mbar_wait(&empty_bar[st], ph ^ 1, status)) break;
-                const int rb = static_cast<int>(t % sh.tiles_r);
-                const int j = static_cast<int>(t / sh.tiles_r);
+                const int k = job_of(jobs, t);
+                const TcShape& sh = jobs.sh[k];
+                const long long tl = t - jobs.tile0[k];
+                const int rb = static_cast<int>(tl % sh.tiles_r);
+                const int j = static_cast<int>(tl / sh.tiles_r);
                 uint8_t* dst = ring + st * kTileBytes;
                 mbar_arrive_expect_tx(&full_bar[st], kTileBytes);
-                tma_load_2d(dst, &tmap, kTile * j, kTile * rb, &full_bar[st]);
-                tma_load_2d(dst + kHalfBytes, &tmap, kTile * j + 64, kTile * rb, &full_bar[st]);
+                tma_load_2d(dst, &jobs.map[k], kTile * j, kTile * rb, &full_bar[st]);
+                tma_load_2d(dst + kHalfBytes, &jobs.map[k], kTile * j + 64, kTile * rb, &full_bar[st]);
             }
             // drain: wait (bounded) until every stage this CTA filled has been consumed
             for (int k = 0; k < kStagesTc && k < i; ++k) {
@@ -192,7 +227,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
             int i = 0;
-            for (long long t = blockIdx.x; t < sh.tiles; t += gridDim.x, ++i) {
+            for (long long t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
                 const int st = i % kStagesTc;
                 const int acc = i % kEpiGroups;
                 if (!mbar_wait(&full_bar[st], (i / kStagesTc) & 1, status)) break;
@@ -219,14 +254,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int k = 0; k < L - 1; ++k) mid[k] = 0.5f * (__ldg(codebook + k) + __ldg(codebook + k + 1));
         int i = e;
-        for (long long t = blockIdx.x + static_cast<long long>(e) * gridDim.x; t < sh.tiles;
+        for (long long t = blockIdx.x + static_cast<long long>(e) * gridDim.x; t < ntiles;
              t += static_cast<long long>(kEpiGroups) * gridDim.x, i += kEpiGroups) {
             // warp-uniform decision: the TMEM loads below are .sync.aligned
             const bool ok = __all_sync(kFullMask, mbar_wait(&tfull_bar[e], (i / kEpiGroups) & 1, status));
             if (!ok) break;
             tc_fence_after();
             const uint32_t taddr = tbase + (static_cast<uint32_t>(quad * 32) << 16) + e * kTile;
-            const long long rb = t % sh.tiles_r, j = t / sh.tiles_r;
+            const int k = job_of(jobs, t);
+            const TcShape& sh = jobs.sh[k];
+            const long long tl = t - jobs.tile0[k];
+            const long long rb = tl % sh.tiles_r, j = tl / sh.tiles_r;
             const long long row = rb * kTile + m;
             const long long gid = row * sh.g_eff + j;
             // pass 1: the squared norm of the rotated group (32 TMEM columns at a time,
@@ -285,11 +323,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty_bar[e]);
             if (row >= sh.r_eff) continue;
-            uint4* dst = reinterpret_cast<uint4*>(packed + gid * (16 * B));
+            uint4* dst = reinterpret_cast<uint4*>(jobs.packed[k] + gid * (16 * B));
 #pragma unroll
             for (int p = 0; p < B; ++p)
                 dst[p] = make_uint4(words[4 * p], words[4 * p + 1], words[4 * p + 2], words[4 * p + 3]);
-            norms[gid] = __half_as_ushort(__float2half_rn(sqrtf(ss * 0.0078125f)));
+            jobs.norms[k][gid] = __half_as_ushort(__float2half_rn(sqrtf(ss * 0.0078125f)));
         }
     }
 
@@ -301,9 +339,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
 }
 
-template <int B, int L>
-cudaError_t launch_tc(const CUtensorMap& map, const TcShape& ts, const float* cb, uint8_t* packed,
-                      uint16_t* norms, unsigned* status, cudaStream_t st) {
+template <int B, int L, int NJ>
+cudaError_t launch_tc(const TcJobs<NJ>& jobs, const float* cb, unsigned* status, cudaStream_t st) {
     const int smem = (1 + kStagesTc) * kTileBytes + 1024;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -311,14 +348,54 @@ cudaError_t launch_tc(const CUtensorMap& map, const TcShape& ts, const float* cb
     static unsigned long long configured = 0;
     const unsigned long long bit = 1ull << (dev & 63);
     if (!(configured & bit)) {
-        e = cudaFuncSetAttribute(quantize_tc_kernel<B, L>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        e = cudaFuncSetAttribute(quantize_tc_kernel<B, L, NJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         configured |= bit;
     }
-    const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(ts.tiles, sm_count())));
-    return launch_pdl(quantize_tc_kernel<B, L>, dim3(grid), dim3(kTcThreads), smem, st, map, ts, cb,
-                      packed, norms, status);
+    const long long ntiles = jobs.tile0[jobs.n];
+    const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(ntiles, sm_count())));
+    return launch_pdl(quantize_tc_kernel<B, L, NJ>, dim3(grid), dim3(kTcThreads), smem, st, jobs, cb, status);
 }
+
+// Shape, tensor map and outputs of one tensor as job k of `jobs`.
+template <int NJ>
+bool add_job(TcJobs<NJ>& jobs, int k, const void* w, const Shape& sh, uint8_t* packed, uint16_t* norms) {
+    const bool flat = sh.cols % kTile == 0;
+    TcShape ts;
+    ts.r_eff = flat ? sh.total_groups : sh.rows;
+    const long long c_eff = flat ? kTile : sh.cols;
+    ts.g_eff = flat ? 1 : sh.groups_per_row;
+    ts.tiles_r = (ts.r_eff + kTile - 1) / kTile;
+    ts.tiles = ts.tiles_r * ts.g_eff;
+    const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(c_eff), static_cast<cuuint64_t>(ts.r_eff)};
+    const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(c_eff) * 2};
+    const cuuint32_t box[2] = {64, kTile};
+    const cuuint32_t estride[2] = {1, 1};
+    const CUresult r = tensor_map_encoder()(&jobs.map[k], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(w),
+                                            gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return false;
+    jobs.sh[k] = ts;
+    jobs.packed[k] = packed;
+    jobs.norms[k] = norms;
+    jobs.tile0[k + 1] = jobs.tile0[k] + ts.tiles;
+    return true;
+}
+
+template <int NJ>
+cudaError_t launch_bits(int bits, const TcJobs<NJ>& jobs, const float* cb, unsigned* status, cudaStream_t st) {
+    switch (bits) {
+        case CQ_BITS_TERNARY: return launch_tc<2, 3, NJ>(jobs, cb, status, st);
+        case 2: return launch_tc<2, 4, NJ>(jobs, cb, status, st);
+        case 3: return launch_tc<3, 8, NJ>(jobs, cb, status, st);
+        default: return launch_tc<4, 16, NJ>(jobs, cb, status, st);
+    }
+}
+
+// Jobs per batched launch: the job list travels in the kernel parameters (at most 32 KB).
+constexpr int kBatchJobs = 128;
+static_assert(sizeof(TcJobs<kBatchJobs>) < 32000, "kernel parameter space");
 
 }  // namespace
 
@@ -333,30 +410,30 @@ bool quantize_tc_supported(int w_dtype, const Shape& sh) {
 cudaError_t launch_quantize_tc(const void* w, const Shape& sh, int bits, const float* codebook,
                                uint8_t* packed, uint16_t* norms, unsigned* status,
                                cudaStream_t stream) {
-    const bool flat = sh.cols % kTile == 0;
-    TcShape ts;
-    ts.r_eff = flat ? sh.total_groups : sh.rows;
-    const long long c_eff = flat ? kTile : sh.cols;
-    ts.g_eff = flat ? 1 : sh.groups_per_row;
-    ts.tiles_r = (ts.r_eff + kTile - 1) / kTile;
-    ts.tiles = ts.tiles_r * ts.g_eff;
+    TcJobs<1> jobs;
+    jobs.n = 1;
+    jobs.tile0[0] = 0;
+    if (!add_job(jobs, 0, w, sh, packed, norms)) return cudaErrorInvalidValue;
+    return launch_bits(bits, jobs, codebook, status, stream);
+}
 
-    CUtensorMap map;
-    const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(c_eff), static_cast<cuuint64_t>(ts.r_eff)};
-    const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(c_eff) * 2};
-    const cuuint32_t box[2] = {64, kTile};
-    const cuuint32_t estride[2] = {1, 1};
-    const CUresult r = tensor_map_encoder()(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(w), gdim,
-                                   gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    switch (bits) {
-        case CQ_BITS_TERNARY: return launch_tc<2, 3>(map, ts, codebook, packed, norms, status, stream);
-        case 2: return launch_tc<2, 4>(map, ts, codebook, packed, norms, status, stream);
-        case 3: return launch_tc<3, 8>(map, ts, codebook, packed, norms, status, stream);
-        default: return launch_tc<4, 16>(map, ts, codebook, packed, norms, status, stream);
+cudaError_t launch_quantize_tc_batch(const QuantizeItem* items, int count, int bits,
+                                     const float* codebook, unsigned* status, cudaStream_t stream) {
+    static TcJobs<kBatchJobs> jobs;  // host staging (large); calls are serialised below
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i0 = 0; i0 < count; i0 += kBatchJobs) {
+        const int n = std::min(kBatchJobs, count - i0);
+        jobs.n = n;
+        jobs.tile0[0] = 0;
+        for (int k = 0; k < n; ++k) {
+            const QuantizeItem& it = items[i0 + k];
+            if (!add_job(jobs, k, it.w, it.sh, it.packed, it.norms)) return cudaErrorInvalidValue;
+        }
+        const cudaError_t e = launch_bits(bits, jobs, codebook, status, stream);
+        if (e != cudaSuccess) return e;
     }
+    return cudaSuccess;
 }
 
 }  // namespace cq

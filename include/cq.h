@@ -144,6 +144,32 @@ int cq_quantize(const void* w, int w_dtype, long long rows, long long cols, int 
                 unsigned short* norms_out, void* stream);
 
 /*
+ * cq_quantize_batch -- cq_quantize over a list of tensors in as few launches as possible.
+ *
+ * Same arithmetic and results as calling cq_quantize on every job in order on `stream`
+ * (same w_dtype, bits, group size and codebook for all).  Quantising a whole model is this
+ * call: the tensors are processed together, so no launch waits for the previous tensor's
+ * last tile.  Because the jobs run concurrently, no job's outputs may overlap another job's
+ * input or outputs.
+ *
+ *   jobs        HOST array of `count` descriptors, read during the call only; each job
+ *               follows cq_quantize's rules for w, rows, cols, packed_out and norms_out
+ *   count       >= 0 (0: nothing to do)
+ * Every job is validated before anything is launched; the first failing job's status is
+ * returned.  Returns CQ_OK after enqueueing.
+ */
+typedef struct cq_quantize_job {
+    const void* w;
+    long long rows;
+    long long cols;
+    unsigned char* packed_out;
+    unsigned short* norms_out;
+} cq_quantize_job;
+
+int cq_quantize_batch(const cq_quantize_job* jobs, int count, int w_dtype, int bits,
+                      int group_size, const float* codebook, void* stream);
+
+/*
  * cq_dequantize -- reconstruct W_hat from packed indices and fp16 norms.
  *
  * Page "Cactus Quants CQ2-bit Quantization", "The CQ2-bit Implementation Pipeline"
@@ -160,6 +186,29 @@ int cq_quantize(const void* w, int w_dtype, long long rows, long long cols, int 
 int cq_dequantize(const unsigned char* packed, const unsigned short* norms, long long rows,
                   long long cols, int bits, int group_size, const float* codebook, void* out,
                   int out_dtype, void* stream);
+
+/*
+ * cq_dequantize_batch -- cq_dequantize over a list of tensors in as few launches as
+ * possible.  Same results as calling cq_dequantize on every job in order on `stream` (same
+ * bits, group size, codebook and out_dtype for all).  The jobs run concurrently, so no job's
+ * output may overlap another job's inputs or output.
+ *
+ *   jobs        HOST array of `count` descriptors, read during the call only; each job
+ *               follows cq_dequantize's rules for packed, norms, rows, cols and out
+ *   count       >= 0 (0: nothing to do)
+ * Every job is validated before anything is launched; the first failing job's status is
+ * returned.  Returns CQ_OK after enqueueing.
+ */
+typedef struct cq_dequantize_job {
+    const unsigned char* packed;
+    const unsigned short* norms;
+    long long rows;
+    long long cols;
+    void* out;
+} cq_dequantize_job;
+
+int cq_dequantize_batch(const cq_dequantize_job* jobs, int count, int bits, int group_size,
+                        const float* codebook, int out_dtype, void* stream);
 
 /*
  * cq_dequant_gemv -- y = W_hat x without materialising W_hat.

@@ -269,6 +269,72 @@ def test_more_than_2g_elements_sampled(ora):
     parity.check_dequant_bf16(to_np(out[torch.from_numpy(sel).to(DEV)]), ref, cols, "2G deq")
 
 
+# shapes for the batched calls: flat, row-tiled, CUDA-core (cols % 8 != 0), tiny and empty
+BATCH_SHAPES = [(256, 512), (37, 1000), (64, 100), (1, 128), (300, 4096), (5, 8), (0, 128),
+                (129, 256), (3, 11008)]
+
+
+def batch_tensor(rows, cols, dtype, seed, tid, sigma):
+    if rows * cols == 0:
+        return torch.empty((rows, cols), dtype=dtype, device=DEV)
+    return dev_tensor(rows, cols, dtype, seed, tid, sigma)
+
+
+@pytest.mark.parametrize("bits", [0, 2, 4])
+def test_quantize_batch_equals_single_calls(ora, bits):
+    """One cq_quantize_batch over assorted shapes returns exactly the bytes of one cq_quantize
+    per tensor; the single calls are the ones checked against the oracle elsewhere, and one
+    batched job is also checked against the oracle here."""
+    ws = [batch_tensor(r, c, torch.bfloat16, 21, k, 0.02) for k, (r, c) in enumerate(BATCH_SHAPES)]
+    got = cq.quantize_batch(ws, bits)
+    for w, (pb, nb) in zip(ws, got):
+        ps, ns = cq.quantize(w, bits)
+        assert torch.equal(pb, ps) and torch.equal(nb.view(torch.int16), ns.view(torch.int16))
+    w_np = to_np(ws[1])
+    o_packed, o_norms, u = ora.quantize(w_np, bits, want_u=True)
+    parity.check_indices(to_np(got[1][0]), o_packed, u, bits, cq.codebook(bits), "batch job 1")
+    parity.check_norms(to_np(got[1][1]), o_norms, parity.group_norms(parity.bf16_to_f64(w_np), 1000))
+
+
+def test_quantize_batch_many_jobs_and_fp32():
+    """More jobs than one launch carries (chunked launches), and an fp32 batch (CUDA-core
+    path for every job)."""
+    shapes = [(3 + (k % 5), 128 * (1 + k % 3)) for k in range(150)]
+    ws = [dev_tensor(r, c, torch.bfloat16, 22, k, 0.02) for k, (r, c) in enumerate(shapes)]
+    got = cq.quantize_batch(ws, 2)
+    for w, (pb, nb) in zip(ws, got):
+        ps, ns = cq.quantize(w, 2)
+        assert torch.equal(pb, ps) and torch.equal(nb.view(torch.int16), ns.view(torch.int16))
+    wf = [batch_tensor(r, c, torch.float32, 23, k, 1.0) for k, (r, c) in enumerate(BATCH_SHAPES)]
+    got = cq.quantize_batch(wf, 3)
+    for w, (pb, nb) in zip(wf, got):
+        ps, ns = cq.quantize(w, 3)
+        assert torch.equal(pb, ps) and torch.equal(nb.view(torch.int16), ns.view(torch.int16))
+
+
+@pytest.mark.parametrize("bits", [0, 2, 3, 4])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_dequantize_batch_equals_single_calls(bits, out_dtype):
+    ws = [batch_tensor(r, c, torch.bfloat16, 24, k, 0.02) for k, (r, c) in enumerate(BATCH_SHAPES)]
+    q = cq.quantize_batch(ws, bits)
+    items = [(pk, nm, r, c) for (pk, nm), (r, c) in zip(q, BATCH_SHAPES)]
+    got = cq.dequantize_batch(items, bits, out_dtype=out_dtype)
+    for (pk, nm, r, c), ob in zip(items, got):
+        os_ = cq.dequantize(pk, nm, r, c, bits, out_dtype=out_dtype)
+        assert ob.shape == (r, c) and torch.equal(ob.view(-1).view(torch.int16 if out_dtype == torch.bfloat16 else torch.int32),
+                                                 os_.view(-1).view(torch.int16 if out_dtype == torch.bfloat16 else torch.int32))
+
+
+def test_dequantize_batch_many_jobs():
+    shapes = [(2 + (k % 7), 128 * (1 + k % 4)) for k in range(140)]
+    ws = [dev_tensor(r, c, torch.bfloat16, 25, k, 0.02) for k, (r, c) in enumerate(shapes)]
+    q = cq.quantize_batch(ws, 2)
+    items = [(pk, nm, r, c) for (pk, nm), (r, c) in zip(q, shapes)]
+    got = cq.dequantize_batch(items, 2)
+    for (pk, nm, r, c), ob in zip(items, got):
+        assert torch.equal(ob.view(torch.int16), cq.dequantize(pk, nm, r, c, 2).view(torch.int16))
+
+
 def test_zz_no_kernel_wait_gave_up():
     """Every bounded wait inside the tensor-core kernels completed during this module."""
     assert cq.device_status() == 0

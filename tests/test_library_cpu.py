@@ -140,6 +140,56 @@ def test_gemv_rejects(L):
     assert g(A, A, 4, 256, 2, 32, None, A, 1, A, A, ws, None) == 2
 
 
+def _qjobs(*jobs):
+    arr = (cq._QuantizeJob * max(1, len(jobs)))()
+    for k, j in enumerate(jobs):
+        arr[k] = cq._QuantizeJob(*j)
+    return ctypes.cast(arr, ctypes.c_void_p), arr
+
+
+def _dqjobs(*jobs):
+    arr = (cq._DequantizeJob * max(1, len(jobs)))()
+    for k, j in enumerate(jobs):
+        arr[k] = cq._DequantizeJob(*j)
+    return ctypes.cast(arr, ctypes.c_void_p), arr
+
+
+def test_quantize_batch_rejects_before_launching(L):
+    q = L.cq_quantize_batch
+    good = (A, 4, 128, A, A)
+    p, _k = _qjobs(good, good)
+    assert q(p, -1, 1, 2, 128, None, None) == 1                 # negative count
+    assert q(None, 1, 1, 2, 128, None, None) == 1               # no job array
+    assert q(p, 2, 2, 2, 128, None, None) == 1                  # bad dtype
+    assert q(p, 2, 1, 1, 128, None, None) == 1                  # bits 1
+    assert q(p, 2, 1, 2, 64, None, None) == 2                   # valid but unsupported group
+    p, _k = _qjobs(good, (A, -1, 128, A, A))
+    assert q(p, 2, 1, 2, 128, None, None) == 1                  # second job: negative rows
+    p, _k = _qjobs(good, (A, 4, 128, None, A))
+    assert q(p, 2, 1, 2, 128, None, None) == 1                  # second job: null packed
+    p, _k = _qjobs((A + 8, 4, 128, A, A), good)
+    assert q(p, 2, 1, 2, 128, None, None) == 4                  # first job misaligned
+    assert q(None, 0, 1, 2, 128, None, None) == 0               # nothing to do
+    p, _k = _qjobs((None, 0, 128, None, None), (None, 7, 0, None, None))
+    assert q(p, 2, 1, 2, 128, None, None) == 0                  # only empty jobs
+
+
+def test_dequantize_batch_rejects_before_launching(L):
+    d = L.cq_dequantize_batch
+    good = (A, A, 4, 128, A)
+    p, _k = _dqjobs(good, good)
+    assert d(p, -1, 2, 128, None, 1, None) == 1
+    assert d(None, 2, 2, 128, None, 1, None) == 1
+    assert d(p, 2, 2, 128, None, 3, None) == 1                  # bad out dtype
+    assert d(p, 2, 6, 128, None, 1, None) == 1                  # bits 6
+    p, _k = _dqjobs(good, (A, None, 4, 128, A))
+    assert d(p, 2, 2, 128, None, 1, None) == 1                  # null norms
+    p, _k = _dqjobs(good, (A, A, 4, 128, A + 4))
+    assert d(p, 2, 2, 128, None, 1, None) == 4                  # misaligned out
+    p, _k = _dqjobs((None, None, 0, 64, None))
+    assert d(p, 1, 3, 128, None, 1, None) == 0                  # only an empty job
+
+
 def test_binding_refuses_cpu_tensors(L):
     torch = pytest.importorskip("torch")
     with pytest.raises(ValueError):
