@@ -67,20 +67,18 @@ struct DqJobs {
     int n;
 };
 
+
+// Job of the tiles a loop visits in increasing order: a cursor that only moves forward.
 template <int NJ>
-__device__ __forceinline__ int job_of(const DqJobs<NJ>& jb, long long t) {
-    if constexpr (NJ == 1) {
-        return 0;
-    } else {
-        int lo = 0, hi = jb.n - 1;  // largest k with tile0[k] <= t
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (jb.tile0[mid] <= t) lo = mid;
-            else hi = mid - 1;
+struct JobCursor {
+    int k = 0;
+    __device__ __forceinline__ int at(const DqJobs<NJ>& jb, long long t) {
+        if constexpr (NJ > 1) {
+            while (t >= jb.tile0[k + 1]) ++k;
         }
-        return lo;
+        return k;
     }
-}
+};
 
 // Element of the group held by MMA column k.
 template <int B>
@@ -192,8 +190,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         fence_mbar_init();
         // the first tiles' codes and norms of this CTA into L2 while the previous kernel finishes
         long long t = blockIdx.x;
+        JobCursor<NJ> cur;
         for (int i = 0; i < kStagesDq && t < ntiles; ++i, t += gridDim.x) {
-            const int k = job_of(jobs, t);
+            const int k = cur.at(jobs, t);
             const DqShape& sh = jobs.sh[k];
             const long long g0 = (t - jobs.tile0[k]) * kTile;
             const long long n = sh.total - g0 < kTile ? sh.total - g0 : kTile;
@@ -243,10 +242,11 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         // ---------------- bulk-copy producer ----------------
         if (lane == 0) {
             int i = 0;
+            JobCursor<NJ> cur;
             for (long long t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
                 const int st = i % kStagesDq;
                 if (!mbar_wait(&empty_bar[st], ((i / kStagesDq) & 1) ^ 1, status)) break;
-                const int k = job_of(jobs, t);
+                const int k = cur.at(jobs, t);
                 const DqShape& sh = jobs.sh[k];
                 const long long g0 = (t - jobs.tile0[k]) * kTile;
                 const long long n = sh.total - g0 < kTile ? sh.total - g0 : kTile;
@@ -290,9 +290,10 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
         const uint32_t a_hi = tbase + lane_off + e * kSlotCols, a_lo = a_hi + 64, d = a_hi + 128;
         int i = e;
+        JobCursor<NJ> cur;
         for (long long t = blockIdx.x + static_cast<long long>(e) * gridDim.x; t < ntiles;
              t += 2LL * gridDim.x, i += 2) {
-            const int k = job_of(jobs, t);
+            const int k = cur.at(jobs, t);
             const DqShape& sh = jobs.sh[k];
             const long long tl = t - jobs.tile0[k];
             const int st = i % kStagesDq;

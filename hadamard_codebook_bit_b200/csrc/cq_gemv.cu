@@ -398,16 +398,9 @@ __global__ void __maxnreg__(96)
 
     // Nothing is read before the dependency wait: loads issued earlier by a programmatic
     // dependent (even of buffers written by kernels that ran before step 1) returned stale
-    // data on this hardware.  The early launch still hides the launch latency, and the codes
-    // of this warp's rows are pulled into L2 meanwhile (L2 is the point of coherence).
+    // data on this hardware.  The early launch still hides the launch latency.  (An L2
+    // prefetch of the codes here measured ~1 us slower per call.)
     pdl_trigger();
-    if (lane < 16 && je > jb) {
-        const long long r = r0 + (lane & 7) + 8 * (lane >> 3);
-        if (r < rows)
-            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(packed + (r * G + jb) * GemvWarp<B>::kBlk),
-                         "r"(static_cast<uint32_t>(je - jb) * GemvWarp<B>::kBlk)
-                         : "memory");
-    }
     pdl_wait();
     float inv_scale;
     load_tables<B>(table, st.tb, inv_scale);

@@ -64,21 +64,18 @@ struct TcJobs {
     int n;
 };
 
-// Job of global tile t (largest k with tile0[k] <= t).
+
+// Job of the tiles a loop visits in increasing order: a cursor that only moves forward.
 template <int NJ>
-__device__ __forceinline__ int job_of(const TcJobs<NJ>& jb, long long t) {
-    if constexpr (NJ == 1) {
-        return 0;
-    } else {
-        int lo = 0, hi = jb.n - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (jb.tile0[mid] <= t) lo = mid;
-            else hi = mid - 1;
+struct JobCursor {
+    int k = 0;
+    __device__ __forceinline__ int at(const TcJobs<NJ>& jb, long long t) {
+        if constexpr (NJ > 1) {
+            while (t >= jb.tile0[k + 1]) ++k;
         }
-        return lo;
+        return k;
     }
-}
+};
 
 // Byte offset of element (row, k) of a 128 x 128 bf16 K-major tile stored as two 64-column
 // halves, each with the 128-byte swizzle (16-byte chunk index XOR row % 8).
@@ -183,8 +180,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         fence_mbar_init();
         // the first tiles of this CTA into L2 while the previous kernel finishes
         long long t = blockIdx.x;
+        JobCursor<NJ> cur;
         for (int i = 0; i < kStagesTc && t < ntiles; ++i, t += gridDim.x) {
-            const int k = job_of(jobs, t);
+            const int k = cur.at(jobs, t);
             const TcShape& sh = jobs.sh[k];
             const long long tl = t - jobs.tile0[k];
             const int rb = static_cast<int>(tl % sh.tiles_r), j = static_cast<int>(tl / sh.tiles_r);
@@ -203,11 +201,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // ---------------- TMA producer ----------------
         if (lane == 0) {
             int i = 0;
+            JobCursor<NJ> cur;
             for (long long t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
                 const int st = i % kStagesTc;
                 const uint32_t ph = (i / kStagesTc) & 1;
                 if (!mbar_wait(&empty_bar[st], ph ^ 1, status)) break;
-                const int k = job_of(jobs, t);
+                const int k = cur.at(jobs, t);
                 const TcShape& sh = jobs.sh[k];
                 const long long tl = t - jobs.tile0[k];
                 const int rb = static_cast<int>(tl % sh.tiles_r);
@@ -254,6 +253,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int k = 0; k < L - 1; ++k) mid[k] = 0.5f * (__ldg(codebook + k) + __ldg(codebook + k + 1));
         int i = e;
+        JobCursor<NJ> cur;
         for (long long t = blockIdx.x + static_cast<long long>(e) * gridDim.x; t < ntiles;
              t += static_cast<long long>(kEpiGroups) * gridDim.x, i += kEpiGroups) {
             // warp-uniform decision: the TMEM loads below are .sync.aligned
@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (!ok) break;
             tc_fence_after();
             const uint32_t taddr = tbase + (static_cast<uint32_t>(quad * 32) << 16) + e * kTile;
-            const int k = job_of(jobs, t);
+            const int k = cur.at(jobs, t);
             const TcShape& sh = jobs.sh[k];
             const long long tl = t - jobs.tile0[k];
             const long long rb = tl % sh.tiles_r, j = tl / sh.tiles_r;
