@@ -30,7 +30,7 @@ _STATUS = {0: "CQ_OK", 1: "CQ_ERR_INVALID_ARG", 2: "CQ_ERR_UNSUPPORTED", 3: "CQ_
 EXPORTS = ("cq_status_string", "cq_version", "cq_device_status", "cq_codebook", "cq_packed_bytes",
            "cq_norm_bytes", "cq_quantize", "cq_dequantize", "cq_dequant_gemv",
            "cq_gemv_workspace_bytes", "cq_dequant_gemv_static", "cq_quantize_batch",
-           "cq_dequantize_batch")
+           "cq_dequantize_batch", "cq_dequant_gemv_batch")
 
 
 class CQError(RuntimeError):
@@ -68,6 +68,7 @@ def lib() -> ctypes.CDLL:
         L.cq_dequant_gemv_static.argtypes = [P, P, ll, ll, i, i, P, P, i, P, P]
         L.cq_quantize_batch.argtypes = [P, i, i, i, i, P, P]
         L.cq_dequantize_batch.argtypes = [P, i, i, i, P, i, P]
+        L.cq_dequant_gemv_batch.argtypes = [P, i, i, i, P, P]
         _lib = L
     return _lib
 
@@ -242,6 +243,45 @@ def dequantize_batch(items, bits: int, group_size: int = GROUP_SIZE, codebook=No
                                          group_size, _cb_ptr(codebook, dev), dt, _stream(dev)),
                "cq_dequantize_batch")
     return outs
+
+
+class _GemvJob(ctypes.Structure):  # cq_gemv_job
+    _fields_ = [("packed", ctypes.c_void_p), ("norms", ctypes.c_void_p), ("rows", ctypes.c_longlong),
+                ("cols", ctypes.c_longlong), ("x", ctypes.c_void_p), ("batch", ctypes.c_int),
+                ("y", ctypes.c_void_p), ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+
+
+def dequant_gemv_batch(items, bits: int, group_size: int = GROUP_SIZE, codebook=None,
+                       workspaces=None, ys=None):
+    """cq_dequant_gemv_batch on a list of (packed, norms, rows, cols, x) on one device ->
+    list of y [batch, rows] fp32.  `workspaces` / `ys`, if given, are lists of tensors (each
+    job needs its own workspace)."""
+    torch = _torch()
+    if not items:
+        return []
+    dev = items[0][0].device
+    jobs = (_GemvJob * len(items))()
+    out = []
+    keep = []  # every job's workspace stays allocated until the launches are enqueued
+    for k, (packed, norms, rows, cols, x) in enumerate(items):
+        if x.dim() == 1:
+            x = x.unsqueeze(0)
+        if x.dtype != torch.bfloat16 or norms.dtype != torch.float16:
+            raise ValueError("x must be bfloat16 and norms float16")
+        batch = x.shape[0]
+        y = ys[k] if ys is not None else torch.empty((batch, rows), dtype=torch.float32, device=dev)
+        wsb = gemv_workspace_bytes(cols, batch)
+        ws = workspaces[k] if workspaces is not None else torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+        keep.append(ws)
+        jobs[k] = _GemvJob(_dev_ptr(packed, "packed"), _dev_ptr(norms, "norms"), rows, cols,
+                           _dev_ptr(x, "x"), batch, _dev_ptr(y, "y"), _dev_ptr(ws, "workspace"),
+                           ws.numel() * ws.element_size())
+        out.append(y)
+    with torch.cuda.device(dev):
+        _check(lib().cq_dequant_gemv_batch(ctypes.cast(jobs, ctypes.c_void_p), len(items), bits,
+                                           group_size, _cb_ptr(codebook, dev), _stream(dev)),
+               "cq_dequant_gemv_batch")
+    return out
 
 
 def dequantize(packed, norms, rows: int, cols: int, bits: int, group_size: int = GROUP_SIZE,

@@ -311,6 +311,50 @@ int cq_dequantize_batch(const cq_dequantize_job* jobs, int count, int bits, int 
     return CQ_OK;
 }
 
+int cq_dequant_gemv_batch(const cq_gemv_job* jobs, int count, int bits, int group_size,
+                          const float* codebook, void* stream) {
+    if (count < 0 || (count > 0 && !jobs)) return CQ_ERR_INVALID_ARG;
+    bool any = false;
+    for (int i = 0; i < count; ++i) {
+        const cq_gemv_job& j = jobs[i];
+        if (j.batch < 1 || j.batch > 8) return CQ_ERR_INVALID_ARG;
+        const int rc = cq::check_common(j.rows, j.cols, bits, group_size);
+        if (rc != CQ_OK) return rc;
+        if (j.rows == 0) continue;
+        if (!j.y) return CQ_ERR_INVALID_ARG;
+        if (!cq::aligned16(j.y)) return CQ_ERR_ALIGNMENT;
+        any = true;
+        if (j.cols == 0) continue;
+        if (!j.packed || !j.norms || !j.x) return CQ_ERR_INVALID_ARG;
+        if (!j.workspace || j.workspace_bytes < cq::gemv_workspace_bytes(j.cols, j.batch))
+            return CQ_ERR_WORKSPACE;
+        if (!cq::aligned16(j.packed) || !cq::aligned16(j.norms) || !cq::aligned16(j.x) ||
+            !cq::aligned16(j.workspace))
+            return CQ_ERR_ALIGNMENT;
+    }
+    if (!any) return CQ_OK;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    std::vector<cq::GemvItem> items;
+    for (int i = 0; i < count; ++i) {
+        const cq_gemv_job& j = jobs[i];
+        if (j.rows == 0) continue;
+        if (j.cols == 0) {  // empty inner dimension: y = 0
+            const cudaError_t e = cudaMemsetAsync(j.y, 0, sizeof(float) * static_cast<size_t>(j.batch) *
+                                                              static_cast<size_t>(j.rows), st);
+            if (e != cudaSuccess) return CQ_ERR_CUDA;
+            continue;
+        }
+        items.push_back({j.packed, j.norms, cq::make_shape(j.rows, j.cols),
+                         static_cast<const uint16_t*>(j.x), j.batch, j.y, j.workspace});
+    }
+    if (items.empty()) return CQ_OK;
+    const float* cb = nullptr;
+    const int rc = cq::resolve_codebook(bits, codebook, &cb);
+    if (rc != CQ_OK) return rc;
+    const cudaError_t e = cq::launch_dequant_gemv_batch(items.data(), static_cast<int>(items.size()), bits, cb, st);
+    return e == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
+}
+
 size_t cq_gemv_workspace_bytes(long long cols, int batch) {
     if (cols < 0 || batch < 1 || batch > 8) return 0;
     return cq::gemv_workspace_bytes(cols, batch);

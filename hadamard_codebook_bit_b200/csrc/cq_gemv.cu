@@ -31,6 +31,7 @@
 //   3/4-bit:  e = 32 t + 4 s + q  (four adjacent codes: one 12- or 16-bit field, spread to
 //             nibble selectors, looked up with byte permutes in 8 / 16-entry byte tables).
 #include <algorithm>
+#include <mutex>
 
 #include "cq_device.cuh"
 #include "cq_internal.h"
@@ -46,8 +47,8 @@ constexpr int kBatchCols = 8;     // MMA N: batch columns, zero padded
 constexpr int kXEntry = 8;        // bytes of B fragment per lane per k-step (4 fp16)
 
 // Workspace: [G][4 k-step pairs][32 lanes] of 8 fp16 | fp32 exponents [G][8] | codeword table.
-size_t frag_bytes(long long G) { return static_cast<size_t>(G) * 8 * 32 * kXEntry; }
-size_t scale_bytes(long long G) { return static_cast<size_t>(G) * kBatchCols * sizeof(float); }
+__host__ __device__ inline size_t frag_bytes(long long G) { return static_cast<size_t>(G) * 8 * 32 * kXEntry; }
+__host__ __device__ inline size_t scale_bytes(long long G) { return static_cast<size_t>(G) * kBatchCols * sizeof(float); }
 
 struct CodeTable {
     uint32_t lo, hi;      // low / high bytes of the fp16 codewords 0..3 (2-bit codes)
@@ -82,18 +83,59 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// The products of one launch (one for cq_dequant_gemv, up to kGemvBatch for the batched
+// call).  Job k owns rotation blocks [group0[k], group0[k + 1]) (one per group) and GEMV blocks
+// [block0[k], block0[k + 1]) (one per 16 rows); its workspace holds x~ fragments, exponents and
+// the codeword table in that order.
+template <int NJ>
+struct GemvJobs {
+    const uint16_t* x[NJ];
+    const uint8_t* packed[NJ];
+    const uint16_t* norms[NJ];
+    char* ws[NJ];
+    float* y[NJ];
+    long long rows[NJ];
+    long long cols[NJ];
+    int G[NJ];
+    int batch[NJ];
+    long long group0[NJ + 1];
+    long long block0[NJ + 1];
+    int n;
+};
+
+// Largest k < n with prefix[k] <= v (v < prefix[n]).
+template <int NJ>
+__device__ __forceinline__ int find_job(const long long (&prefix)[NJ + 1], int n, long long v) {
+    if constexpr (NJ == 1) {
+        return 0;
+    } else {
+        int lo = 0, hi = n - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (prefix[mid] <= v) lo = mid;
+            else hi = mid - 1;
+        }
+        return lo;
+    }
+}
+
 // ---------------------------------------------------------------------------------------
 // step 1: rotate the activations into fragment order (+ codeword table)
 // ---------------------------------------------------------------------------------------
 
-template <int B, int L>
+template <int B, int L, int NJ>
 __global__ void __launch_bounds__(kRotThreads)
-    rotate_x_kernel(const uint16_t* __restrict__ x, long long cols, long long G, int batch,
-                    const float* __restrict__ codebook, __half* __restrict__ xfrag,
-                    float* __restrict__ xscale, CodeTable* __restrict__ table) {
+    rotate_x_kernel(const __grid_constant__ GemvJobs<NJ> jobs, const float* __restrict__ codebook) {
     pdl_trigger();  // the GEMV may be scheduled now; it waits for this kernel before any access
     pdl_wait();
-    const long long j = blockIdx.x;
+    const int jk = find_job<NJ>(jobs.group0, jobs.n, blockIdx.x);
+    const long long j = blockIdx.x - jobs.group0[jk];
+    const uint16_t* __restrict__ x = jobs.x[jk];
+    const long long cols = jobs.cols[jk], G = jobs.G[jk];
+    const int batch = jobs.batch[jk];
+    __half* __restrict__ xfrag = reinterpret_cast<__half*>(jobs.ws[jk]);
+    float* __restrict__ xscale = reinterpret_cast<float*>(jobs.ws[jk] + frag_bytes(G));
+    CodeTable* __restrict__ table = reinterpret_cast<CodeTable*>(jobs.ws[jk] + frag_bytes(G) + scale_bytes(G));
     const int b = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (j == 0 && threadIdx.x < 32) {
@@ -366,16 +408,23 @@ struct GemvWarp {
     }
 };
 
-template <int B>
+template <int B, int NJ>
 __global__ void __maxnreg__(96)
-    gemv_split_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ norms,
-                      long long rows, int G, const uint4* xfrag, const float2* xscale,
-                      const CodeTable* table, int batch, float* __restrict__ y) {
+    gemv_split_kernel(const __grid_constant__ GemvJobs<NJ> jobs) {
     __shared__ float4 red[kMaxSplit][32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int S = static_cast<int>(blockDim.x >> 5);
     const int g = lane >> 2, t = lane & 3;
-    const long long r0 = static_cast<long long>(blockIdx.x) * kRowsPerBlock;
+    const int jk = find_job<NJ>(jobs.block0, jobs.n, blockIdx.x);
+    const uint8_t* __restrict__ packed = jobs.packed[jk];
+    const uint16_t* __restrict__ norms = jobs.norms[jk];
+    const long long rows = jobs.rows[jk];
+    const int G = jobs.G[jk], batch = jobs.batch[jk];
+    float* __restrict__ y = jobs.y[jk];
+    const uint4* xfrag = reinterpret_cast<const uint4*>(jobs.ws[jk]);
+    const float2* xscale = reinterpret_cast<const float2*>(jobs.ws[jk] + frag_bytes(G));
+    const CodeTable* table = reinterpret_cast<const CodeTable*>(jobs.ws[jk] + frag_bytes(G) + scale_bytes(G));
+    const long long r0 = (blockIdx.x - jobs.block0[jk]) * kRowsPerBlock;
     const long long ra = r0 + g, rb = r0 + g + 8;
     const bool oka = ra < rows, okb = rb < rows;
 
@@ -431,20 +480,21 @@ __global__ void __maxnreg__(96)
     if (okb && c1 < batch) y[c1 * rows + rb] = a.w * f;
 }
 
-// Registers per thread of gemv_split_kernel<B> on the current device (queried once).
-template <int B>
+// Registers per thread of gemv_split_kernel<B, NJ> on the current device (queried once).
+template <int B, int NJ>
 int gemv_regs() {
     static int regs = 0;
     if (regs == 0) {
         cudaFuncAttributes fa;
-        regs = (cudaFuncGetAttributes(&fa, gemv_split_kernel<B>) == cudaSuccess && fa.numRegs > 0) ? fa.numRegs : 128;
+        regs = (cudaFuncGetAttributes(&fa, gemv_split_kernel<B, NJ>) == cudaSuccess && fa.numRegs > 0) ? fa.numRegs : 128;
     }
     return regs;
 }
 
 // Warps per block.  The row blocks are spread over the SMs in one round when they fit:
 // every SM holds ceil(blocks / SMs) of them, and the split is the largest (up to 16 warps,
-// at least two groups a warp) for which that many blocks stay resident by registers.
+// at least two groups a warp of the narrowest job) for which that many blocks stay resident
+// by registers.
 int gemv_split(long long blocks, long long G, int regs) {
     const long long sms = sm_count();
     const long long per_sm = (blocks + sms - 1) / sms;
@@ -457,24 +507,47 @@ int gemv_split(long long blocks, long long G, int regs) {
     return best;
 }
 
-template <int B>
-cudaError_t launch_gemv_bits(const uint8_t* packed, const uint16_t* norms, const Shape& sh,
-                             const uint4* xfrag, const float2* xscale, const CodeTable* table,
-                             int batch, float* y, cudaStream_t st) {
-    const long long blocks = (sh.rows + kRowsPerBlock - 1) / kRowsPerBlock;
-    const int split = gemv_split(blocks, sh.groups_per_row, gemv_regs<B>());
-    return launch_pdl(gemv_split_kernel<B>, dim3(static_cast<unsigned>(blocks)), dim3(32 * split), 0, st,
-                      packed, norms, sh.rows, static_cast<int>(sh.groups_per_row), xfrag, xscale,
-                      table, batch, y);
+template <int B, int L, int NJ>
+cudaError_t launch_pair(const GemvJobs<NJ>& jobs, const float* codebook, cudaStream_t st) {
+    long long min_g = jobs.G[0];
+    for (int k = 1; k < jobs.n; ++k) min_g = std::min<long long>(min_g, jobs.G[k]);
+    const long long groups = jobs.group0[jobs.n], blocks = jobs.block0[jobs.n];
+    cudaError_t e = launch_pdl(rotate_x_kernel<B, L, NJ>, dim3(static_cast<unsigned>(groups)),
+                               dim3(kRotThreads), 0, st, jobs, codebook);
+    if (e != cudaSuccess) return e;
+    const int split = gemv_split(blocks, min_g, gemv_regs<B, NJ>());
+    return launch_pdl(gemv_split_kernel<B, NJ>, dim3(static_cast<unsigned>(blocks)), dim3(32 * split), 0, st,
+                      jobs);
 }
 
-template <int B, int L>
-cudaError_t launch_rotate(const uint16_t* x, const Shape& sh, int batch, const float* codebook,
-                          __half* xfrag, float* xscale, CodeTable* table, cudaStream_t st) {
-    return launch_pdl(rotate_x_kernel<B, L>, dim3(static_cast<unsigned>(sh.groups_per_row)),
-                      dim3(kRotThreads), 0, st, x, sh.cols, sh.groups_per_row, batch, codebook,
-                      xfrag, xscale, table);
+template <int NJ>
+cudaError_t launch_jobs(int bits, const GemvJobs<NJ>& jobs, const float* codebook, cudaStream_t st) {
+    switch (bits) {
+        case CQ_BITS_TERNARY: return launch_pair<2, 3, NJ>(jobs, codebook, st);
+        case 2: return launch_pair<2, 4, NJ>(jobs, codebook, st);
+        case 3: return launch_pair<3, 8, NJ>(jobs, codebook, st);
+        default: return launch_pair<4, 16, NJ>(jobs, codebook, st);
+    }
 }
+
+template <int NJ>
+void set_job(GemvJobs<NJ>& jobs, int k, const GemvItem& it) {
+    jobs.x[k] = it.x;
+    jobs.packed[k] = it.packed;
+    jobs.norms[k] = it.norms;
+    jobs.ws[k] = static_cast<char*>(it.workspace);
+    jobs.y[k] = it.y;
+    jobs.rows[k] = it.sh.rows;
+    jobs.cols[k] = it.sh.cols;
+    jobs.G[k] = static_cast<int>(it.sh.groups_per_row);
+    jobs.batch[k] = it.batch;
+    jobs.group0[k + 1] = jobs.group0[k] + it.sh.groups_per_row;
+    jobs.block0[k + 1] = jobs.block0[k] + (it.sh.rows + kRowsPerBlock - 1) / kRowsPerBlock;
+}
+
+// Products per batched launch pair: the job list travels in the kernel parameters.
+constexpr int kGemvBatch = 256;
+static_assert(sizeof(GemvJobs<kGemvBatch>) < 32000, "kernel parameter space");
 
 }  // namespace
 
@@ -488,28 +561,27 @@ size_t gemv_workspace_bytes(long long cols, int batch) {
 cudaError_t launch_dequant_gemv(const uint8_t* packed, const uint16_t* norms, const Shape& sh,
                                 int bits, const float* codebook, const uint16_t* x, int batch,
                                 float* y, void* workspace, cudaStream_t stream) {
-    const long long G = sh.groups_per_row;
-    char* ws = static_cast<char*>(workspace);
-    __half* xfrag = reinterpret_cast<__half*>(ws);
-    float* xscale = reinterpret_cast<float*>(ws + frag_bytes(G));
-    CodeTable* table = reinterpret_cast<CodeTable*>(ws + frag_bytes(G) + scale_bytes(G));
-    const uint4* xf = reinterpret_cast<const uint4*>(xfrag);
-    const float2* xs = reinterpret_cast<const float2*>(xscale);
-    cudaError_t e;
-    switch (bits) {
-        case CQ_BITS_TERNARY:
-            e = launch_rotate<2, 3>(x, sh, batch, codebook, xfrag, xscale, table, stream);
-            return e != cudaSuccess ? e : launch_gemv_bits<2>(packed, norms, sh, xf, xs, table, batch, y, stream);
-        case 2:
-            e = launch_rotate<2, 4>(x, sh, batch, codebook, xfrag, xscale, table, stream);
-            return e != cudaSuccess ? e : launch_gemv_bits<2>(packed, norms, sh, xf, xs, table, batch, y, stream);
-        case 3:
-            e = launch_rotate<3, 8>(x, sh, batch, codebook, xfrag, xscale, table, stream);
-            return e != cudaSuccess ? e : launch_gemv_bits<3>(packed, norms, sh, xf, xs, table, batch, y, stream);
-        default:
-            e = launch_rotate<4, 16>(x, sh, batch, codebook, xfrag, xscale, table, stream);
-            return e != cudaSuccess ? e : launch_gemv_bits<4>(packed, norms, sh, xf, xs, table, batch, y, stream);
+    GemvJobs<1> jobs;
+    jobs.n = 1;
+    jobs.group0[0] = jobs.block0[0] = 0;
+    set_job(jobs, 0, GemvItem{packed, norms, sh, x, batch, y, workspace});
+    return launch_jobs(bits, jobs, codebook, stream);
+}
+
+cudaError_t launch_dequant_gemv_batch(const GemvItem* items, int count, int bits,
+                                      const float* codebook, cudaStream_t stream) {
+    static GemvJobs<kGemvBatch> jobs;  // host staging (large); calls are serialised below
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i0 = 0; i0 < count; i0 += kGemvBatch) {
+        const int n = std::min(kGemvBatch, count - i0);
+        jobs.n = n;
+        jobs.group0[0] = jobs.block0[0] = 0;
+        for (int k = 0; k < n; ++k) set_job(jobs, k, items[i0 + k]);
+        const cudaError_t e = launch_jobs(bits, jobs, codebook, stream);
+        if (e != cudaSuccess) return e;
     }
+    return cudaSuccess;
 }
 
 }  // namespace cq

@@ -81,6 +81,16 @@ struct DequantizeItem {
     void* out;
 };
 
+struct GemvItem {
+    const uint8_t* packed;
+    const uint16_t* norms;
+    Shape sh;
+    const uint16_t* x;
+    int batch;
+    float* y;
+    void* workspace;
+};
+
 // Tensor-core quantiser (cq_quantize_tc.cu): bf16 input, cols % 8 == 0.
 bool quantize_tc_supported(int w_dtype, const Shape& s);
 cudaError_t launch_quantize_tc(const void* w, const Shape& s, int bits, const float* codebook,
@@ -110,5 +120,8 @@ size_t gemv_workspace_bytes(long long cols, int batch);
 cudaError_t launch_dequant_gemv(const uint8_t* packed, const uint16_t* norms, const Shape& s,
                                 int bits, const float* codebook, const uint16_t* x, int batch,
                                 float* y, void* workspace, cudaStream_t stream);
+// Several products (none with rows == 0 or cols == 0) in as few launches as possible.
+cudaError_t launch_dequant_gemv_batch(const GemvItem* items, int count, int bits,
+                                      const float* codebook, cudaStream_t stream);
 
 }  // namespace cq

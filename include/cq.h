@@ -244,6 +244,34 @@ int cq_dequant_gemv(const unsigned char* packed, const unsigned short* norms, lo
                     const void* x, int batch, float* y, void* workspace,
                     size_t workspace_bytes, void* stream);
 
+/*
+ * cq_dequant_gemv_batch -- several independent cq_dequant_gemv products in one rotation
+ * launch and one GEMV launch.  Same results as calling cq_dequant_gemv on every job in order
+ * on `stream` (same bits, group size and codebook for all): the products run concurrently,
+ * so no job's y or workspace may overlap anything another job reads or writes.
+ *
+ *   jobs        HOST array of `count` descriptors, read during the call only; each job
+ *               follows cq_dequant_gemv's rules for its fields (its own workspace of at least
+ *               cq_gemv_workspace_bytes(cols, batch) bytes)
+ *   count       >= 0 (0: nothing to do)
+ * Every job is validated before anything is launched; the first failing job's status is
+ * returned.  Returns CQ_OK after enqueueing.
+ */
+typedef struct cq_gemv_job {
+    const unsigned char* packed;
+    const unsigned short* norms;
+    long long rows;
+    long long cols;
+    const void* x;
+    int batch;
+    float* y;
+    void* workspace;
+    size_t workspace_bytes;
+} cq_gemv_job;
+
+int cq_dequant_gemv_batch(const cq_gemv_job* jobs, int count, int bits, int group_size,
+                          const float* codebook, void* stream);
+
 /* Workspace bytes cq_dequant_gemv needs for this cols and batch (0 if invalid or cols == 0). */
 size_t cq_gemv_workspace_bytes(long long cols, int batch);
 

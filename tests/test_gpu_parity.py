@@ -335,6 +335,47 @@ def test_dequantize_batch_many_jobs():
         assert torch.equal(ob.view(torch.int16), cq.dequantize(pk, nm, r, c, 2).view(torch.int16))
 
 
+@pytest.mark.parametrize("bits", [0, 2, 4])
+def test_gemv_batch_matches_oracle(ora, bits):
+    """cq_dequant_gemv_batch over assorted products (ragged, several batch sizes, empty rows,
+    empty inner dimension) against the oracle, and repeatable bit for bit."""
+    shapes = [(37, 1000, 3), (256, 4096, 1), (64, 128, 8), (1, 129, 2), (0, 256, 1), (5, 0, 2),
+              (300, 11008, 1)]
+    items, refs = [], []
+    for k, (r, c, b) in enumerate(shapes):
+        w = batch_tensor(r, c, torch.bfloat16, 26, k, 0.02)
+        pk, nm = cq.quantize(w, bits)
+        x = batch_tensor(b, c, torch.bfloat16, 27, k, 1.0)
+        items.append((pk, nm, r, c, x))
+    ys = cq.dequant_gemv_batch(items, bits)
+    ys2 = cq.dequant_gemv_batch(items, bits)
+    torch.cuda.synchronize()
+    for (pk, nm, r, c, x), y, y2 in zip(items, ys, ys2):
+        assert y.shape == (x.shape[0], r) and torch.equal(y, y2)
+        if r == 0:
+            continue
+        if c == 0:
+            assert torch.all(y == 0)
+            continue
+        ref = ora.dequant_gemv(to_np(pk), to_np(nm), r, c, bits, to_np(x))
+        parity.check_gemv(to_np(y), ref, f"gemv batch {r}x{c} b={x.shape[0]}")
+
+
+def test_gemv_batch_many_jobs(ora):
+    """More products than one launch pair carries."""
+    items = []
+    for k in range(260):
+        r, c = 3 + k % 5, 128 * (1 + k % 3)
+        pk, nm = cq.quantize(dev_tensor(r, c, torch.bfloat16, 28, k, 0.02), 2)
+        items.append((pk, nm, r, c, dev_tensor(1, c, torch.bfloat16, 29, k, 1.0)))
+    ys = cq.dequant_gemv_batch(items, 2)
+    torch.cuda.synchronize()
+    for k in (0, 1, 128, 255, 256, 259):
+        pk, nm, r, c, x = items[k]
+        ref = ora.dequant_gemv(to_np(pk), to_np(nm), r, c, 2, to_np(x))
+        parity.check_gemv(to_np(ys[k]), ref, f"gemv batch job {k}")
+
+
 def test_zz_no_kernel_wait_gave_up():
     """Every bounded wait inside the tensor-core kernels completed during this module."""
     assert cq.device_status() == 0

@@ -190,6 +190,31 @@ def test_dequantize_batch_rejects_before_launching(L):
     assert d(p, 1, 3, 128, None, 1, None) == 0                  # only an empty job
 
 
+def test_gemv_batch_rejects_before_launching(L):
+    g = L.cq_dequant_gemv_batch
+    ws = cq.gemv_workspace_bytes(256, 1)
+
+    def jobs(*js):
+        arr = (cq._GemvJob * len(js))()
+        for k, j in enumerate(js):
+            arr[k] = cq._GemvJob(*j)
+        return ctypes.cast(arr, ctypes.c_void_p), arr
+
+    good = (A, A, 4, 256, A, 1, A, A, ws)
+    p, _k = jobs(good, good)
+    assert g(p, -1, 2, 128, None, None) == 1
+    assert g(None, 2, 2, 128, None, None) == 1
+    assert g(p, 2, 5, 128, None, None) == 1                          # bits 5
+    p, _k = jobs(good, (A, A, 4, 256, A, 9, A, A, ws))
+    assert g(p, 2, 2, 128, None, None) == 1                          # batch 9
+    p, _k = jobs(good, (A, A, 4, 256, A, 1, A, A, ws - 1))
+    assert g(p, 2, 2, 128, None, None) == 5                          # workspace too small
+    p, _k = jobs(good, (A, A, 4, 256, A, 1, A + 4, A, ws))
+    assert g(p, 2, 2, 128, None, None) == 4                          # misaligned y
+    p, _k = jobs((None, None, 0, 256, None, 1, None, None, 0))
+    assert g(p, 1, 2, 128, None, None) == 0                          # rows == 0: nothing to do
+
+
 def test_binding_refuses_cpu_tensors(L):
     torch = pytest.importorskip("torch")
     with pytest.raises(ValueError):
