@@ -621,31 +621,44 @@ def run_reference_arm(args):
 
 
 def run_ncu_case(args):
-    """Small fixed launches for a detailed ncu capture: a 32768x4096 bf16 tensor (256 MiB,
-    larger than L2) quantised and dequantised, then one 11008x4096 2-bit GEMV at batch 1
-    and 8.  Each kernel launches 1 + 3 times (the first is a warm-up)."""
+    """Small fixed launches for a detailed ncu capture, in the form the bench step uses them:
+    eight 4096x4096 bf16 tensors (256 MiB, larger than L2) through cq_quantize_batch,
+    cq_dequantize_batch and a batch-1 cq_dequant_gemv_batch, then one 11008x4096 2-bit
+    cq_dequant_gemv at batch 1 and 8.  Each call runs 1 + 3 times (the first is a warm-up)."""
     import torch
     import hadamard_codebook_bit_b200 as cq
     import synth
     device = torch.device("cuda:0")
-    rows, cols, bits = 32768, 4096, args.ncu_bits
-    w = torch.empty((rows, cols), dtype=torch.bfloat16, device=device)
-    synth.fill_normal_(w, 3, 0, 0.02)
-    packed, norms = cq.empty_packed(rows, cols, bits, device)
-    out = torch.empty_like(w)
+    n_t, rows, cols, bits = 8, 4096, 4096, args.ncu_bits
+    ws = []
+    for k in range(n_t):
+        w = torch.empty((rows, cols), dtype=torch.bfloat16, device=device)
+        synth.fill_normal_(w, 3, k, 0.02)
+        ws.append(w)
+    outs = [cq.empty_packed(rows, cols, bits, device) for _ in range(n_t)]
+    deq = [torch.empty_like(w) for w in ws]
     for _ in range(4):
-        cq.quantize(w, bits, out=(packed, norms))
+        cq.quantize_batch(ws, bits, outs=outs)
+    items = [(pk, nm, rows, cols) for pk, nm in outs]
     for _ in range(4):
-        cq.dequantize(packed, norms, rows, cols, bits, out=out)
-    g_rows, g_cols = 11008, 4096
-    pk, nm = cq.quantize(w.view(-1)[:g_rows * g_cols].view(g_rows, g_cols), 2)
-    for batch in (1, 8):
-        x = torch.empty((batch, g_cols), dtype=torch.bfloat16, device=device)
-        synth.fill_normal_(x, 4, 100, 1.0)
+        cq.dequantize_batch(items, bits, outs=deq)
+    x = torch.empty((1, cols), dtype=torch.bfloat16, device=device)
+    synth.fill_normal_(x, 4, 100, 1.0)
+    if bits in (0, 2):
+        g_items = [(pk, nm, rows, cols, x) for pk, nm in outs]
         for _ in range(4):
-            cq.dequant_gemv(pk, nm, g_rows, g_cols, 2, x)
+            cq.dequant_gemv_batch(g_items, bits)
+    g_rows, g_cols = 11008, 4096
+    wg = torch.empty((g_rows, g_cols), dtype=torch.bfloat16, device=device)
+    synth.fill_normal_(wg, 4, 0, 0.02)
+    pk, nm = cq.quantize(wg, 2)
+    for batch in (1, 8):
+        xb = torch.empty((batch, g_cols), dtype=torch.bfloat16, device=device)
+        synth.fill_normal_(xb, 4, 100, 1.0)
+        for _ in range(4):
+            cq.dequant_gemv(pk, nm, g_rows, g_cols, 2, xb)
     torch.cuda.synchronize(device)
-    print(json.dumps({"ncu_case": "done", "rows": rows, "cols": cols, "bits": bits}))
+    print(json.dumps({"ncu_case": "done", "tensors": n_t, "rows": rows, "cols": cols, "bits": bits}))
 
 
 def main():
