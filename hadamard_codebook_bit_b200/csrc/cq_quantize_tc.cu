@@ -135,6 +135,53 @@ __device__ __forceinline__ uint32_t pack2_signbits(const float (&v)[32], const f
     return w;
 }
 
+// --- 3/4-bit nearest codeword through a warp-held bucket table ---------------------------
+// In normalised units u = r / n the decision thresholds are the fixed codebook midpoints m_k.
+// u is mapped monotonically onto 32 buckets (t = sat(u sA + 1/2), bucket = rint(31 t)); lane b
+// holds bucket b's entry: the bits of the one midpoint falling in that bucket (or a huge
+// finite value) with the number of midpoints below the bucket in the low 4 mantissa bits.  The
+// index is then  base + [u > threshold]  after one shuffle.  Clearing the low mantissa bits
+// moves a threshold by at most 15 ulp, far inside the 1e-5 decision tolerance.  If a bucket
+// would hold two midpoints (a crowded custom codebook) the select tree is used instead.
+struct BucketLookup {
+    uint32_t entry;
+    float sA;
+    bool ok;
+};
+
+__device__ __forceinline__ uint32_t bucket_of(float u, float sA) {
+    const float t = __saturatef(fmaf(u, sA, 0.5f));
+    return __float_as_uint(fmaf(t, 31.0f, 12582912.0f)) & 31u;  // 1.5 * 2^23: rint in the low bits
+}
+
+template <int L>
+__device__ __forceinline__ BucketLookup make_buckets(const float (&mid)[L - 1], int lane) {
+    BucketLookup bl;
+    float span = fmaxf(fabsf(mid[0]), fabsf(mid[L - 2])) * 1.1f;
+    if (!(span > 0.0f)) span = 1.0f;
+    bl.sA = 0.5f / span;
+    uint32_t thr = 0x7f7ffff0u, base = 0u;
+    int cnt = 0;
+#pragma unroll
+    for (int k = 0; k < L - 1; ++k) {
+        const uint32_t b = bucket_of(mid[k], bl.sA);
+        if (b < static_cast<uint32_t>(lane)) {
+            ++base;
+        } else if (b == static_cast<uint32_t>(lane)) {
+            thr = __float_as_uint(mid[k]) & ~15u;
+            ++cnt;
+        }
+    }
+    bl.entry = thr | base;
+    bl.ok = !__any_sync(kFullMask, cnt > 1);
+    return bl;
+}
+
+__device__ __forceinline__ uint32_t bucket_index(float u, const BucketLookup& bl) {
+    const uint32_t e = __shfl_sync(kFullMask, bl.entry, static_cast<int>(bucket_of(u, bl.sA)));
+    return (e & 15u) + (u > __uint_as_float(e) ? 1u : 0u);
+}
+
 template <int B, int L, int NJ>
 __global__ void __launch_bounds__(kTcThreads, 1)
     quantize_tc_kernel(const __grid_constant__ TcJobs<NJ> jobs, const float* __restrict__ codebook,
@@ -252,6 +299,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         float mid[L - 1];
 #pragma unroll
         for (int k = 0; k < L - 1; ++k) mid[k] = 0.5f * (__ldg(codebook + k) + __ldg(codebook + k + 1));
+        BucketLookup bl{0u, 1.0f, false};
+        if constexpr (B != 2) bl = make_buckets<L>(mid, lane);
         int i = e;
         JobCursor<NJ> cur;
         for (long long t = blockIdx.x + static_cast<long long>(e) * gridDim.x; t < ntiles;
@@ -280,6 +329,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             const float ss = (ps[0] + ps[1]) + (ps[2] + ps[3]);
             const float nrm = sqrtf(ss);
+            const float inv_n = nrm > 0.0f ? __frcp_rn(nrm) : 0.0f;  // u = r / n (0 for a zero group)
             float T[L - 1];
 #pragma unroll
             for (int k = 0; k < L - 1; ++k) T[k] = nrm > 0.0f ? mid[k] * nrm : mid[k];
@@ -300,22 +350,43 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 } else if constexpr (B == 3) {
 #pragma unroll
                     for (int w = 0; w < B; ++w) words[B * c + w] = 0u;
+                    if (bl.ok) {
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) {
-                        const uint32_t idx = nearest_index<L>(v[q], T);
-                        const int bit = B * q, w = B * c + (bit >> 5), sh2 = bit & 31;
-                        words[w] |= idx << sh2;
-                        if (sh2 + B > 32) words[w + 1] |= idx >> (32 - sh2);
+                        for (int q = 0; q < 32; ++q) {
+                            const uint32_t idx = bucket_index(v[q] * inv_n, bl);
+                            const int bit = B * q, w = B * c + (bit >> 5), sh2 = bit & 31;
+                            words[w] |= idx << sh2;
+                            if (sh2 + B > 32) words[w + 1] |= idx >> (32 - sh2);
+                        }
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) {
+                            const uint32_t idx = nearest_index<L>(v[q], T);
+                            const int bit = B * q, w = B * c + (bit >> 5), sh2 = bit & 31;
+                            words[w] |= idx << sh2;
+                            if (sh2 + B > 32) words[w + 1] |= idx >> (32 - sh2);
+                        }
                     }
                 } else {
                     // 32 / B fields per word, accumulated top-down: word = (word << B) + idx
+                    if (bl.ok) {
 #pragma unroll
-                    for (int w = 0; w < B; ++w) {
-                        uint32_t acc = 0u;
+                        for (int w = 0; w < B; ++w) {
+                            uint32_t acc = 0u;
 #pragma unroll
-                        for (int q = 32 / B - 1; q >= 0; --q)
-                            acc = (acc << B) + nearest_index<L>(v[w * (32 / B) + q], T);
-                        words[B * c + w] = acc;
+                            for (int q = 32 / B - 1; q >= 0; --q)
+                                acc = (acc << B) + bucket_index(v[w * (32 / B) + q] * inv_n, bl);
+                            words[B * c + w] = acc;
+                        }
+                    } else {
+#pragma unroll
+                        for (int w = 0; w < B; ++w) {
+                            uint32_t acc = 0u;
+#pragma unroll
+                            for (int q = 32 / B - 1; q >= 0; --q)
+                                acc = (acc << B) + nearest_index<L>(v[w * (32 / B) + q], T);
+                            words[B * c + w] = acc;
+                        }
                     }
                 }
             }
