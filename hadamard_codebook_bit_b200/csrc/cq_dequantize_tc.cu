@@ -237,6 +237,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     }
     const float inv_scale = ldexpf(1.0f, -cs) * kInvSqrt128;
     __syncthreads();  // tab_s
+    // the same table held one entry per lane, repeated every 2^B lanes, so that a shuffle whose
+    // index is the code plus any higher bits (only the low 5 bits of the index count) reads it
+    const uint32_t tab_lane = tab_s[lane & ((1 << B) - 1) & 15];
 
     if (warp == 0) {
         // ---------------- bulk-copy producer ----------------
@@ -336,21 +339,27 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                         }
                     }
                 } else {
+                    static_assert(L == (1 << B), "3/4-bit codebooks use every code");
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
                         const int e0 = 64 * half + 2 * c;  // elements e0, e0 + 1
-                        uint32_t code[2];
+                        uint32_t t[2];
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
+                            // the code sits in the low B bits; bits above it are ignored by the
+                            // lane-repeated table
                             const int bit = B * (e0 + u);
                             const uint32_t lo = wd[bit >> 5];
-                            const uint32_t hi = ((bit >> 5) + 1 < 4 * B) ? wd[(bit >> 5) + 1] : 0u;
-                            uint32_t cd = __funnelshift_r(lo, hi, bit & 31) & ((1u << B) - 1u);
-                            code[u] = cd < static_cast<uint32_t>(L) ? cd : static_cast<uint32_t>(L - 1);
+                            uint32_t idx;
+                            if ((bit & 31) + B <= 32) {
+                                idx = lo >> (bit & 31);
+                            } else {
+                                idx = __funnelshift_r(lo, wd[(bit >> 5) + 1], bit & 31);
+                            }
+                            t[u] = __shfl_sync(kFullMask, tab_lane, static_cast<int>(idx));
                         }
-                        const uint32_t t0 = tab_s[code[0]], t1 = tab_s[code[1]];
-                        rh[c] = prmt(t0, t1, 0x5410u);
-                        rl[c] = prmt(t0, t1, 0x7632u);
+                        rh[c] = prmt(t[0], t[1], 0x5410u);
+                        rl[c] = prmt(t[0], t[1], 0x7632u);
                     }
                 }
                 tmem_st32(a_hi + 32 * half, rh);

@@ -216,6 +216,24 @@ def test_custom_codebook(ora):
     roundtrip_check(ora, w_dev, 2, "custom codebook", codebook=cb)
 
 
+@pytest.mark.parametrize("bits", [3, 4])
+def test_custom_codebook_wide_levels(ora, bits):
+    """A caller codebook with evenly spread levels: the bucket-table search handles it."""
+    cb = np.linspace(-0.25, 0.21, 1 << bits).astype(np.float32)
+    w_dev = dev_tensor(96, 1024, torch.bfloat16, 30, bits, 0.02)
+    roundtrip_check(ora, w_dev, bits, f"wide codebook {bits}-bit", codebook=cb)
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+def test_custom_codebook_crowded_levels(ora, bits):
+    """Two midpoints closer than a bucket: the quantiser falls back to the select tree."""
+    cb = np.linspace(-0.25, 0.21, 1 << bits).astype(np.float32)
+    cb[3] = cb[2] + 1e-4  # levels 2, 3 nearly equal -> midpoints 1|2 and 2|3 share a bucket
+    cb[4] = cb[3] + 2e-4
+    w_dev = dev_tensor(96, 1024, torch.bfloat16, 31, bits, 0.02)
+    roundtrip_check(ora, w_dev, bits, f"crowded codebook {bits}-bit", codebook=cb)
+
+
 def test_unused_ternary_code_decodes_as_top_level(ora):
     packed = torch.full((3, 2, 32), 0xFF, dtype=torch.uint8, device=DEV)  # every code = 3
     norms = torch.full((3, 2), 1.5, dtype=torch.float16, device=DEV)
