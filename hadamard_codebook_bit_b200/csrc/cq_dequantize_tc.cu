@@ -8,16 +8,19 @@
 // 2^cs, is split into two fp16 values hi + lo that sum to it within 2^-22 relative, so two
 // fp16 MMAs with exact +-1 weights and fp32 accumulation give the fp32 result.
 //
-// Persistent kernel, one 320-thread CTA per SM (all 512 TMEM columns):
+// Persistent kernel, one 448-thread CTA per SM (all 512 TMEM columns: A buffers 0-255, D
+// buffers 256-511):
 //   warp 0      bulk-copies each tile's packed blocks (128 groups, contiguous) into a
 //               4-stage shared-memory ring;
-//   warp 1      owns TMEM; one lane issues per tile 16 tcgen05.mma (M=128, N=128, K=16):
-//               8 for the hi plane, 8 for the lo plane, A read from TMEM, B = H_int from
-//               shared memory, into the tile slot's fp32 accumulator;
-//   warps 2-9   two decode/epilogue warpgroups, one TMEM slot each (A hi 64 columns, A lo 64,
-//               D 128), taking alternating tiles: a thread decodes its group's codes into
-//               fp16 pairs with byte permutes, writes them to TMEM (tcgen05.st), and after the
-//               MMAs reads its group's 128 results back, scales them by the norm and stores.
+//   warp 1      one lane issues per tile 16 tcgen05.mma (M=128, N=128, K=16): 8 for the hi
+//               plane, 8 for the lo plane, A read from A buffer i % 2 in TMEM, B = H_int from
+//               shared memory, into D buffer i % 2;
+//   warps 2-5   decode: a thread turns its group's codes into fp16 pairs with byte permutes
+//               (or a lane-held table) and writes them to the A buffer with tcgen05.st;
+//   warps 6-13  two epilogue groups, one per D buffer, taking alternating tiles: a thread
+//               reads its group's 128 results back, scales them by the norm and stores them.
+// Decode, MMA and epilogue of consecutive tiles overlap: A and D buffers are handed over
+// through their own mbarrier pairs.  One launch may cover several tensors (a job list).
 //
 // K order of a 2-bit group.  The MMA contracts over the 128 input elements in any order as
 // long as A and B agree: column k = 16 w + 4 p + q of A holds element e = 16 w + 4 q + p, the
@@ -37,11 +40,12 @@ namespace {
 using namespace dev;
 using namespace sm100;
 
-constexpr int kDqThreads = 64 + 256;
+constexpr int kDqThreads = 64 + 128 + 256;  // producer, MMA, decode group, 2 epilogue groups
 constexpr int kTile = 128;
 constexpr int kStagesDq = 4;
-constexpr int kSlotCols = 256;                  // A hi (64) + A lo (64) + D (128)
-constexpr int kTmemColsDq = 2 * kSlotCols;
+constexpr int kACols = 128;                     // one A buffer: hi plane (64) + lo plane (64)
+constexpr int kDBase = 256;                     // D buffers at columns 256 and 384
+constexpr int kTmemColsDq = 512;
 constexpr int kHBytes = kTile * kTile * 2;      // fp16 H_int, two 64-column swizzled halves
 constexpr int kHHalf = kHBytes / 2;
 constexpr uint32_t kIdescDq = idesc_f16_f32(kTile, kTile);
@@ -146,7 +150,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                          unsigned* __restrict__ status) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full_bar[kStagesDq], empty_bar[kStagesDq];
-    __shared__ __align__(8) uint64_t afull_bar[2], dfull_bar[2];
+    __shared__ __align__(8) uint64_t afull_bar[2], aempty_bar[2], dfull_bar[2], dempty_bar[2];
     __shared__ uint32_t tmem_slot;
     __shared__ uint32_t tab_s[16];  // fp16 (hi | lo << 16) of every code (3- and 4-bit codes)
     constexpr int kStageBytes = kTile * 16 * B;
@@ -184,8 +188,10 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             mbar_init(&empty_bar[s], 4);
         }
         for (int a = 0; a < 2; ++a) {
-            mbar_init(&afull_bar[a], 4);
-            mbar_init(&dfull_bar[a], 1);
+            mbar_init(&afull_bar[a], 4);   // the decode group's four warps
+            mbar_init(&aempty_bar[a], 1);  // MMA completion
+            mbar_init(&dfull_bar[a], 1);   // MMA completion
+            mbar_init(&dempty_bar[a], 4);  // epilogue group a's four warps
         }
         fence_mbar_init();
         // the first tiles' codes and norms of this CTA into L2 while the previous kernel finishes
@@ -267,10 +273,11 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         if (lane == 0) {
             int i = 0;
             for (long long t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
-                const int e = i & 1;
+                const int e = i & 1;  // A buffer and D buffer of this tile
                 if (!mbar_wait(&afull_bar[e], (i >> 1) & 1, status)) break;
+                if (!mbar_wait(&dempty_bar[e], ((i >> 1) & 1) ^ 1, status)) break;
                 tc_fence_after();
-                const uint32_t a_hi = tbase + e * kSlotCols, a_lo = a_hi + 64, d = a_hi + 128;
+                const uint32_t a_hi = tbase + e * kACols, a_lo = a_hi + 64, d = tbase + kDBase + e * kTile;
                 const uint32_t b_base = smem_u32(hmat);
 #pragma unroll
                 for (int k = 0; k < kTile / 16; ++k)
@@ -282,26 +289,29 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                     mma_f16_tmem_a(d, a_lo + 8 * k,
                                    smem_desc_sw128(b_base + (k >> 2) * kHHalf + (k & 3) * 32), kIdescDq,
                                    true);
+                mma_commit(&aempty_bar[e]);
                 mma_commit(&dfull_bar[e]);
             }
         }
-    } else {
-        // ---------------- decode + epilogue ----------------
-        const int e = (warp - 2) >> 2;
+    } else if (warp < 6) {
+        // ---------------- decode: codes -> A buffer (i & 1) ----------------
         const int quad = warp & 3;
         const int m = quad * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-        const uint32_t a_hi = tbase + lane_off + e * kSlotCols, a_lo = a_hi + 64, d = a_hi + 128;
-        int i = e;
+        int i = 0;
         JobCursor<NJ> cur;
-        for (long long t = blockIdx.x + static_cast<long long>(e) * gridDim.x; t < ntiles;
-             t += 2LL * gridDim.x, i += 2) {
+        for (long long t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
             const int k = cur.at(jobs, t);
             const DqShape& sh = jobs.sh[k];
             const long long tl = t - jobs.tile0[k];
             const int st = i % kStagesDq;
+            const int e = i & 1;
+            bool ok = mbar_wait(&full_bar[st], (i / kStagesDq) & 1, status);
+            ok = ok && mbar_wait(&aempty_bar[e], ((i >> 1) & 1) ^ 1, status);
             // the group's four warps decide together whether to go on
-            if (!named_barrier_and(1 + e, 128, mbar_wait(&full_bar[st], (i / kStagesDq) & 1, status))) break;
+            if (!named_barrier_and(1, 128, ok)) break;
+            tc_fence_after();
+            const uint32_t a_hi = tbase + lane_off + e * kACols, a_lo = a_hi + 64;
             const long long gid = tl * kTile + m;
             const bool valid = gid < sh.total;
             uint32_t wd[4 * B];
@@ -316,7 +326,6 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                     wd[4 * v + 3] = u.w;
                 }
             }
-            const float nrm = valid ? __half2float(__ushort_as_half(__ldg(jobs.norms[k] + gid))) : 0.0f;
 
             // A planes: 64 columns each, written 32 at a time
 #pragma unroll
@@ -367,20 +376,37 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             }
             tmem_st_wait();
             tc_fence_before();
-            // the stage's words are consumed (decoded); order these generic reads before the
-            // producer's next bulk write into the stage
+            // the stage's words are consumed; order these generic reads before the producer's
+            // next bulk write into the stage
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&empty_bar[st]);
                 mbar_arrive(&afull_bar[e]);
             }
-
-            const bool leader = (warp == 2 + 4 * e) && lane == 0;
+        }
+    } else {
+        // ---------------- epilogue group e: D buffer e -> W_hat (tiles i = e mod 2) ----------
+        const int e = (warp - 6) >> 2;
+        const int quad = warp & 3;
+        const int m = quad * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+        const uint32_t d = tbase + lane_off + kDBase + e * kTile;
+        const bool leader = (warp == 6 + 4 * e) && lane == 0;
+        int i = e;
+        JobCursor<NJ> cur;
+        for (long long t = blockIdx.x + static_cast<long long>(e) * gridDim.x; t < ntiles;
+             t += 2LL * gridDim.x, i += 2) {
+            const int k = cur.at(jobs, t);
+            const DqShape& sh = jobs.sh[k];
+            const long long tl = t - jobs.tile0[k];
+            const long long gid = tl * kTile + m;
+            const bool valid = gid < sh.total;
+            const float nrm = valid ? __half2float(__ushort_as_half(__ldg(jobs.norms[k] + gid))) : 0.0f;
             bool ok = mbar_wait(&dfull_bar[e], (i >> 1) & 1, status);
             // before the staging tile is rewritten, this group's previous stores have read it
             if (sh.flat && leader) bulk_wait_read0();
-            if (!named_barrier_and(1 + e, 128, ok)) break;
+            if (!named_barrier_and(2 + e, 128, ok)) break;
             tc_fence_after();
             const float scale = nrm * inv_scale;
             constexpr int kPer = kBF16 ? 8 : 4;  // values per 16-byte chunk
@@ -410,8 +436,12 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                         *reinterpret_cast<uint4*>(so + OutTile<kBF16>::chunk_offset(m, (32 * c + off) / kPer)) = o;
                     }
                 }
+                // D buffer read out: the MMAs of the tile after next may overwrite it
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&dempty_bar[e]);
                 fence_proxy_async_smem();
-                named_barrier(1 + e, 128);
+                named_barrier(2 + e, 128);
                 if (leader) {
 #pragma unroll
                     for (int b = 0; b < OutTile<kBF16>::kBoxes; ++b)
@@ -435,9 +465,12 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                             store_chunk<kBF16>(jobs.out[k], base + 32 * c + off, v, off, scale);
                     }
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&dempty_bar[e]);
             }
         }
-        if ((warp == 2 + 4 * e) && lane == 0) bulk_wait0();  // tensor-map stores done before exit
+        if (leader) bulk_wait0();  // tensor-map stores done before exit
     }
 
     tc_fence_before();
