@@ -146,13 +146,28 @@ __global__ void __launch_bounds__(kRotThreads)
         const int k = threadIdx.x < 16 ? (threadIdx.x < L ? static_cast<int>(threadIdx.x) : L - 1) : 0;
         const uint32_t u = __half_as_ushort(__float2half_rn(ldexpf(__ldg(codebook + k), cs)));
         if (threadIdx.x < 16) table->h[threadIdx.x] = static_cast<uint16_t>(u);
-        // bytes of codewords 0..3 gathered in every lane
         uint32_t lo = 0, hi = 0;
+        if constexpr (B == 2) {
+            // 2-bit codes: integer codewords C = rint(c 2^cs) (|C| < 2^14) split as
+            // C = 256 Ch + Cl, Ch in [-64, 64], Cl in [-128, 127]; lo / hi hold the int8
+            // bytes of Ch / Cl for codes 0..3
+            const int cq = __float2int_rn(ldexpf(__ldg(codebook + (threadIdx.x < 4 ? k : 0)), cs));
+            const int ch = (cq + 128) >> 8, cl = cq - (ch << 8);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const uint32_t uq = __shfl_sync(kFullMask, u, q);
-            lo |= (uq & 0xffu) << (8 * q);
-            hi |= (uq >> 8) << (8 * q);
+            for (int q = 0; q < 4; ++q) {
+                const uint32_t hq = static_cast<uint32_t>(__shfl_sync(kFullMask, ch, q)) & 0xffu;
+                const uint32_t lq = static_cast<uint32_t>(__shfl_sync(kFullMask, cl, q)) & 0xffu;
+                lo |= hq << (8 * q);
+                hi |= lq << (8 * q);
+            }
+        } else {
+            // bytes of the fp16 codewords 0..3 gathered in every lane
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint32_t uq = __shfl_sync(kFullMask, u, q);
+                lo |= (uq & 0xffu) << (8 * q);
+                hi |= (uq >> 8) << (8 * q);
+            }
         }
         if (threadIdx.x == 0) {
             table->lo = lo;
@@ -194,11 +209,22 @@ __global__ void __launch_bounds__(kRotThreads)
     // [j][s / 2][lane][8 halves], halves 4 (s % 2) + q
     const int t = lane >> 3;
     if constexpr (B == 2) {
-        const int wsel = (lane >> 2) & 1, q = lane & 3;
+        // 16-bit integer X = rint(x~ 2^-e) = 256 Xh + Xl as two int8 planes, planes h / l of
+        // batch column b being B columns 2 (b % 4), 2 (b % 4) + 1 of n-tile b / 4.  Element e
+        // of the group goes to lane t = e / 32 of k-step s = 2 ((e / 16) % 2) + (e / 8) % 2,
+        // register r = e % 2, byte (e / 2) % 4 (the order in which the GEMV decodes the codes).
+        // Entry layout: [group][n-tile][lane][k-step][r][byte], 32 bytes per lane.
+        uint8_t* xb = reinterpret_cast<uint8_t*>(xfrag);
+        const int nt = b >> 2, nl = 2 * (b & 3);
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            const int s = 4 * wsel + p;
-            xfrag[((j * 4 + (s >> 1)) * 32 + 4 * b + t) * 8 + 4 * (s & 1) + q] = __float2half_rn(v[p] * down);
+        for (int i = 0; i < 4; ++i) {
+            const int e = 4 * lane + i;
+            const int xq = __float2int_rn(v[i] * down);
+            const int xh = (xq + 128) >> 8, xl = xq - (xh << 8);
+            const int t = e >> 5, ks = 2 * ((e >> 4) & 1) + ((e >> 3) & 1), r = e & 1, by = (e >> 1) & 3;
+            const long long o = ((j * 2 + nt) * 32 + 4 * nl + t) * 32 + ks * 8 + 4 * r + by;
+            xb[o] = static_cast<uint8_t>(xh);
+            xb[o + 4 * 32] = static_cast<uint8_t>(xl);  // lane + 4: B column nl + 1
         }
     } else {
         const int s = lane & 7;
@@ -408,6 +434,109 @@ struct GemvWarp {
     }
 };
 
+__device__ __forceinline__ void mma_i8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                       uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// 2-bit codes on the int8 tensor cores.  C = 256 Ch + Cl (codewords) and X = 256 Xh + Xl
+// (rotated activations) are 16-bit integers in two int8 planes each; for a k-step the A
+// operand of plane P is one byte permute of the 4-entry table of P per four codes, with the
+// codes as nibble selectors straight from the packed word (w >> (16 hi + 2 r)) & 0x3333.  B
+// holds Xh and Xl of batch column b in columns 2 (b % 4) and 2 (b % 4) + 1, so lane t's
+// accumulators are the four cross products of batch column t (+ 4 per extra n-tile), combined
+// per group in fp32 as 65536 ChXh + 256 (ChXl + ClXh) + ClXl.
+template <int NT>
+struct GemvWarpI8 {
+    static constexpr int kBlk = 32;
+    static constexpr int kD = NT == 1 ? 8 : 4;  // groups in flight
+    const uint8_t* pa;
+    const uint8_t* pb;
+    const uint16_t* na;
+    const uint16_t* nb;
+    const uint4* xf;   // this lane's 32 bytes of B fragments of n-tile 0 of the current group
+    const float* xs;   // exponents 2^e of the current group (8 columns)
+    bool bcol[NT];     // lane holds a real B column in n-tile nt
+    int t;
+    uint32_t th, tl;   // int8 bytes of Ch / Cl for codes 0..3
+    float tot[NT][2];  // batch column t + 4 nt, rows g and g + 8
+
+    template <bool kFull>
+    __device__ __forceinline__ void batch(int n) {
+        Seg<2> ca[kD], cb[kD];
+        float sa[kD], sb[kD];
+#pragma unroll
+        for (int u = 0; u < kD; ++u) {
+            const bool on = kFull || u < n;
+            ca[u] = load_seg<2>(pa + u * kBlk, t, on);
+            cb[u] = load_seg<2>(pb + u * kBlk, t, on);
+            sa[u] = on ? __half2float(__ushort_as_half(__ldg(na + u))) : 0.0f;
+            sb[u] = on ? __half2float(__ushort_as_half(__ldg(nb + u))) : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < kD; ++u) {
+            if (!kFull && u >= n) break;
+            uint4 bq[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                bq[nt][0] = bq[nt][1] = make_uint4(0, 0, 0, 0);
+                const uint4* p = xf + u * 128 + nt * 64;
+                asm volatile(
+                    "{\n\t.reg .pred q;\n\t"
+                    "setp.ne.u32 q, %8, 0;\n\t"
+                    "@q ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%9];\n\t"
+                    "@q ld.global.nc.v4.u32 {%4, %5, %6, %7}, [%10];\n\t}"
+                    : "+r"(bq[nt][0].x), "+r"(bq[nt][0].y), "+r"(bq[nt][0].z), "+r"(bq[nt][0].w),
+                      "+r"(bq[nt][1].x), "+r"(bq[nt][1].y), "+r"(bq[nt][1].z), "+r"(bq[nt][1].w)
+                    : "r"(static_cast<uint32_t>(bcol[nt])), "l"(p), "l"(p + 1));
+            }
+            float xsv[NT];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(xsv[nt]) : "l"(xs + u * 8 + t + 4 * nt));
+            int ah[NT][4], al[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) ah[nt][q] = al[nt][q] = 0;
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                const int wsel = ks >> 1, sh = 16 * (ks & 1);
+                const uint32_t sa0 = (ca[u].w[wsel] >> sh) & 0x3333u, sa1 = (ca[u].w[wsel] >> (sh + 2)) & 0x3333u;
+                const uint32_t sb0 = (cb[u].w[wsel] >> sh) & 0x3333u, sb1 = (cb[u].w[wsel] >> (sh + 2)) & 0x3333u;
+                const uint32_t h0 = prmt(th, th, sa0), h1 = prmt(th, th, sb0), h2 = prmt(th, th, sa1), h3 = prmt(th, th, sb1);
+                const uint32_t l0 = prmt(tl, tl, sa0), l1 = prmt(tl, tl, sb0), l2 = prmt(tl, tl, sa1), l3 = prmt(tl, tl, sb1);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const uint4& q = bq[nt][ks >> 1];
+                    const uint32_t b0 = (ks & 1) ? q.z : q.x, b1 = (ks & 1) ? q.w : q.y;
+                    mma_i8(ah[nt], h0, h1, h2, h3, b0, b1);
+                    mma_i8(al[nt], l0, l1, l2, l3, b0, b1);
+                }
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const float va = fmaf(static_cast<float>(ah[nt][0]), 65536.0f,
+                                      fmaf(static_cast<float>(ah[nt][1] + al[nt][0]), 256.0f, static_cast<float>(al[nt][1])));
+                const float vb = fmaf(static_cast<float>(ah[nt][2]), 65536.0f,
+                                      fmaf(static_cast<float>(ah[nt][3] + al[nt][2]), 256.0f, static_cast<float>(al[nt][3])));
+                tot[nt][0] = fmaf(sa[u] * xsv[nt], va, tot[nt][0]);
+                tot[nt][1] = fmaf(sb[u] * xsv[nt], vb, tot[nt][1]);
+            }
+        }
+        pa += kD * kBlk;
+        pb += kD * kBlk;
+        na += kD;
+        nb += kD;
+        xf += kD * 128;
+        xs += kD * 8;
+    }
+};
+
 template <int B, int NJ>
 __global__ void __maxnreg__(96)
     gemv_split_kernel(const __grid_constant__ GemvJobs<NJ> jobs) {
@@ -480,6 +609,83 @@ __global__ void __maxnreg__(96)
     if (okb && c1 < batch) y[c1 * rows + rb] = a.w * f;
 }
 
+// 2-bit codes: the same block / split structure as gemv_split_kernel on the int8 path.
+template <int NT, int NJ>
+__global__ void __maxnreg__(96)
+    gemv_i8_kernel(const __grid_constant__ GemvJobs<NJ> jobs) {
+    __shared__ float4 red[kMaxSplit][32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int S = static_cast<int>(blockDim.x >> 5);
+    const int g = lane >> 2, t = lane & 3;
+    const int jk = find_job<NJ>(jobs.block0, jobs.n, blockIdx.x);
+    const uint8_t* __restrict__ packed = jobs.packed[jk];
+    const uint16_t* __restrict__ norms = jobs.norms[jk];
+    const long long rows = jobs.rows[jk];
+    const int G = jobs.G[jk], batch = jobs.batch[jk];
+    float* __restrict__ y = jobs.y[jk];
+    const uint4* xfrag = reinterpret_cast<const uint4*>(jobs.ws[jk]);
+    const float* xscale = reinterpret_cast<const float*>(jobs.ws[jk] + frag_bytes(G));
+    const CodeTable* table = reinterpret_cast<const CodeTable*>(jobs.ws[jk] + frag_bytes(G) + scale_bytes(G));
+    const long long r0 = (blockIdx.x - jobs.block0[jk]) * kRowsPerBlock;
+    const long long ra = r0 + g, rb = r0 + g + 8;
+    const bool oka = ra < rows, okb = rb < rows;
+    const int chunk = (G + S - 1) / S;
+    const int jb = min(G, warp * chunk), je = min(G, jb + chunk);
+
+    GemvWarpI8<NT> st;
+    st.pa = packed + ((oka ? ra : 0) * G + jb) * 32;
+    st.pb = packed + ((okb ? rb : 0) * G + jb) * 32;
+    st.na = norms + (oka ? ra : 0) * G + jb;
+    st.nb = norms + (okb ? rb : 0) * G + jb;
+    st.xf = xfrag + static_cast<long long>(jb) * 128 + 2 * lane;
+    st.xs = xscale + static_cast<long long>(jb) * 8;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        st.bcol[nt] = (g >> 1) + 4 * nt < batch;
+        st.tot[nt][0] = st.tot[nt][1] = 0.0f;
+    }
+    st.t = t;
+
+    // no global access before the dependency wait (see gemv_split_kernel)
+    pdl_trigger();
+    pdl_wait();
+    const uint4 head = ld_v4_volatile(table);  // Ch bytes, Cl bytes, 2^-cs, pad
+    st.th = head.x;
+    st.tl = head.y;
+    const float inv_scale = __uint_as_float(head.z);
+
+    int n = je - jb;
+    constexpr int kD = GemvWarpI8<NT>::kD;
+    for (; n >= kD; n -= kD) st.template batch<true>(n);
+    if (n > 0) st.template batch<false>(n);
+
+    float4 a = make_float4(st.tot[0][0], st.tot[0][1], NT > 1 ? st.tot[NT - 1][0] : 0.0f,
+                           NT > 1 ? st.tot[NT - 1][1] : 0.0f);
+    if (S > 1) {
+        red[warp][lane] = a;
+        __syncthreads();
+        if (warp != 0) return;
+        a = red[0][lane];
+        for (int w = 1; w < S; ++w) {
+            const float4 b = red[w][lane];
+            a.x += b.x;
+            a.y += b.y;
+            a.z += b.z;
+            a.w += b.w;
+        }
+    }
+    const float f = inv_scale * kInvSqrt128;
+    // lane (g, t) holds rows g and g + 8 of batch column t (and t + 4)
+    if (t < batch) {
+        if (oka) y[t * rows + ra] = a.x * f;
+        if (okb) y[t * rows + rb] = a.y * f;
+    }
+    if (NT > 1 && t + 4 < batch) {
+        if (oka) y[(t + 4) * rows + ra] = a.z * f;
+        if (okb) y[(t + 4) * rows + rb] = a.w * f;
+    }
+}
+
 // Registers per thread of gemv_split_kernel<B, NJ> on the current device (queried once).
 template <int B, int NJ>
 int gemv_regs() {
@@ -507,17 +713,42 @@ int gemv_split(long long blocks, long long G, int regs) {
     return best;
 }
 
+template <int NT, int NJ>
+int gemv_i8_regs() {
+    static int regs = 0;
+    if (regs == 0) {
+        cudaFuncAttributes fa;
+        regs = (cudaFuncGetAttributes(&fa, gemv_i8_kernel<NT, NJ>) == cudaSuccess && fa.numRegs > 0) ? fa.numRegs : 128;
+    }
+    return regs;
+}
+
 template <int B, int L, int NJ>
 cudaError_t launch_pair(const GemvJobs<NJ>& jobs, const float* codebook, cudaStream_t st) {
     long long min_g = jobs.G[0];
-    for (int k = 1; k < jobs.n; ++k) min_g = std::min<long long>(min_g, jobs.G[k]);
+    int max_batch = jobs.batch[0];
+    for (int k = 1; k < jobs.n; ++k) {
+        min_g = std::min<long long>(min_g, jobs.G[k]);
+        max_batch = std::max(max_batch, jobs.batch[k]);
+    }
     const long long groups = jobs.group0[jobs.n], blocks = jobs.block0[jobs.n];
     cudaError_t e = launch_pdl(rotate_x_kernel<B, L, NJ>, dim3(static_cast<unsigned>(groups)),
                                dim3(kRotThreads), 0, st, jobs, codebook);
     if (e != cudaSuccess) return e;
-    const int split = gemv_split(blocks, min_g, gemv_regs<B, NJ>());
-    return launch_pdl(gemv_split_kernel<B, NJ>, dim3(static_cast<unsigned>(blocks)), dim3(32 * split), 0, st,
-                      jobs);
+    if constexpr (B == 2) {
+        if (max_batch <= 4) {
+            const int split = gemv_split(blocks, min_g, gemv_i8_regs<1, NJ>());
+            return launch_pdl(gemv_i8_kernel<1, NJ>, dim3(static_cast<unsigned>(blocks)), dim3(32 * split), 0,
+                              st, jobs);
+        }
+        const int split = gemv_split(blocks, min_g, gemv_i8_regs<2, NJ>());
+        return launch_pdl(gemv_i8_kernel<2, NJ>, dim3(static_cast<unsigned>(blocks)), dim3(32 * split), 0, st,
+                          jobs);
+    } else {
+        const int split = gemv_split(blocks, min_g, gemv_regs<B, NJ>());
+        return launch_pdl(gemv_split_kernel<B, NJ>, dim3(static_cast<unsigned>(blocks)), dim3(32 * split), 0,
+                          st, jobs);
+    }
 }
 
 template <int NJ>
