@@ -8,28 +8,32 @@
 //
 // Step 1 (rotate_x_kernel, one block per group j, one warp per batch column b < 8):
 //   x~_bj = H_int x_bj (zero for b >= batch), scaled by 2^-e_bj so its largest magnitude sits
-//   in [2^13, 2^14), rounded to fp16 and written in the register-fragment order of the
-//   tensor-core B operand; the exponents go to an fp32 table.  Block 0 also writes the
-//   codeword table (fp16, one exact power-of-two scale) used by step 2.
+//   in [2^13, 2^14), and written in the register-fragment order of the tensor-core B operand:
+//   for 2-bit codes as a 16-bit integer X = 256 Xh + Xl in two int8 planes, for 3/4-bit codes
+//   rounded to fp16.  The exponents go to an fp32 table.  Block 0 also writes the codeword
+//   table (one exact power-of-two scale): int8 planes Ch, Cl of C = 256 Ch + Cl for 2-bit
+//   codes, fp16 bytes for 3/4-bit codes.
 //
-// Step 2 (gemv_split_kernel, launched as a programmatic dependent of step 1): a block of S
-// warps owns 16 output rows; warp w takes a contiguous chunk of about G / S groups, S chosen
-// so that all row blocks are resident at once.  Per group a lane reads
-// its 32 codes of rows g and g + 8 straight from global memory (one coalesced 8/12/16-byte
-// load per row, four groups in flight at once), decodes them into fp16 A fragments and issues
-// eight m16n8k16 fp16 MMAs (A = codewords of 16 rows x 16 weights, B = x~ of 16 weights x 8
-// columns, fp32 accumulate), folded into fp32 totals as  total += n_rj * 2^e_bj * acc.  The S
-// warps' totals are summed in a fixed order, so the output is deterministic.
+// 2-bit codes (gemv_i8_kernel): m16n8k32 int8 MMAs with exact int32 accumulation per group;
+// the A operand of a plane is one byte permute of a 4-entry table per four codes.  3/4-bit
+// codes (gemv_split_kernel): m16n8k16 fp16 MMAs.  Both are launched as programmatic
+// dependents of step 1 and share one structure: a block of S warps owns 16 output rows; warp
+// w takes a contiguous chunk of about G / S groups, S chosen so that all row blocks are
+// resident at once when they fit.  Per group a lane reads its 32 codes of rows g and g + 8
+// straight from global memory (one coalesced 8/12/16-byte load per row, several groups in
+// flight), builds the A fragments, runs the MMAs against x~, and folds the group's result
+// into fp32 totals as  total += n_rj * 2^e_bj * acc.  The S warps' totals are summed in a
+// fixed order, so the output is deterministic.
 //
-// K order inside a group.  The MMA contracts over the 16 weights of a k-step in any order
-// as long as A and B agree.  Lane (g, t) = (lane / 4, lane % 4) holds codes 32 t .. 32 t + 31
-// of each of its rows; in k-step s its four weights q = 0..3 (MMA k = 2t, 2t+1, 2t+8, 2t+9) are
-//   2-bit:    e = 32 t + 16 (s / 4) + 4 q + s % 4  (the codes at bit 2 (s % 4) of the four
-//             bytes of the lane's word s / 4: decoded with a shift, a mask, two integer
-//             multiply-adds that form byte-permute selectors and two PRMTs from a 4-entry
-//             fp16 table held in two registers);
-//   3/4-bit:  e = 32 t + 4 s + q  (four adjacent codes: one 12- or 16-bit field, spread to
-//             nibble selectors, looked up with byte permutes in 8 / 16-entry byte tables).
+// K order inside a group.  The MMA contracts over the weights of a k-step in any order as
+// long as A and B agree.  Lane (g, t) = (lane / 4, lane % 4) holds codes 32 t .. 32 t + 31 of
+// each of its rows (bits 64 t .. 64 t + 63 of a 2-bit row block).
+//   2-bit (int8, k-step of 32): in k-step s = 2 w + h, register r, byte q the lane takes
+//             e = 32 t + 16 w + 8 h + 2 q + r: the codes that (word w >> (16 h + 2 r)) & 0x3333
+//             places in selector nibbles q = 0..3.
+//   3/4-bit (fp16, k-step of 16): four weights q = 0..3 (MMA k = 2t, 2t+1, 2t+8, 2t+9) are
+//             e = 32 t + 4 s + q: four adjacent codes, one 12- or 16-bit field spread to nibble
+//             selectors and looked up with byte permutes in 8 / 16-entry byte tables.
 #include <algorithm>
 #include <mutex>
 
@@ -63,11 +67,6 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return d;
 }
 
-__device__ __forceinline__ uint32_t mad_hi(uint32_t a, uint32_t b, uint32_t c) {
-    uint32_t d;
-    asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
-}
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
     return static_cast<uint32_t>(__half_as_ushort(__float2half_rn(lo))) |
@@ -270,31 +269,17 @@ __device__ __forceinline__ Seg<B> load_seg(const uint8_t* __restrict__ blk, int 
     return r;
 }
 
-// Byte tables of the fp16 codewords: lo[k] / hi[k] hold the low / high bytes of codes
-// 4k..4k+3.  The 2-bit decode uses lo[0], hi[0] only.
+// Byte tables of the fp16 codewords (3/4-bit codes): lo[k] / hi[k] hold the low / high
+// bytes of codes 4k..4k+3.
 struct ByteTables {
     uint32_t lo[4], hi[4];
 };
 
-// x >> n with the shift on the integer multiply-add unit (n > 0), keeping the ALU free for
-// the masks and byte permutes
-template <int N>
-__device__ __forceinline__ uint32_t shr_mul(uint32_t x) {
-    if constexpr (N == 0) {
-        return x;
-    } else {
-        return mad_hi(x, 1u << (32 - N), 0u);
-    }
-}
-
 // A-fragment registers of one row in k-step S: r0 = (c[k=2t], c[2t+1]), r1 = (c[2t+8], c[2t+9]).
 template <int B, int S>
 __device__ __forceinline__ void decode(const Seg<B>& sg, const ByteTables& tb, uint32_t& r0, uint32_t& r1) {
-    if constexpr (B == 2) {
-        const uint32_t sw = shr_mul<2 * (S & 3)>(sg.w[S >> 2]) & 0x03030303u;  // code q in byte q
-        r0 = prmt(tb.lo[0], tb.hi[0], sw * 0x11u + 0x4040u);                 // codes q = 0, 1
-        r1 = prmt(tb.lo[0], tb.hi[0], mad_hi(sw, 0x110000u, 0x4040u));       // codes q = 2, 3
-    } else {
+    static_assert(B == 3 || B == 4, "2-bit codes take the int8 path");
+    {
         uint32_t sel, m = 0x3210u;
         uint32_t lo4, hi4;
         if constexpr (B == 4) {
@@ -333,10 +318,7 @@ template <int B>
 __device__ __forceinline__ void load_tables(const CodeTable* table, ByteTables& tb, float& inv_scale) {
     const uint4 head = ld_v4_volatile(table);  // lo, hi, inv_scale, pad
     inv_scale = __uint_as_float(head.z);
-    if constexpr (B == 2) {
-        tb.lo[0] = head.x;
-        tb.hi[0] = head.y;
-    } else {
+    {
         const uint4 h0 = ld_v4_volatile(reinterpret_cast<const uint8_t*>(table) + 16);  // h[0..7]
         const uint4 h1 = ld_v4_volatile(reinterpret_cast<const uint8_t*>(table) + 32);  // h[8..15]
         const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};

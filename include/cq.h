@@ -220,11 +220,14 @@ int cq_dequantize_batch(const cq_dequantize_job* jobs, int count, int bits, int 
  * fp32.  The memory-bandwidth motive is page "Performance Differences Between 2-Bit and
  * 4-Bit Quantization in Needle", "Model Size and Memory Bandwidth".
  *
- * Arithmetic: the products run on the tensor cores in fp16 with fp32 accumulation.  The
- * codewords are scaled by one exact power of two per call and each rotated activation
- * group by its own power of two (largest magnitude in [2^13, 2^14)) before rounding to
- * fp16, so any finite input is in range; the relative error of y is about 2e-4 (bound
- * 1e-3 per output vector).  Summation order is fixed: repeated calls give identical bits.
+ * Arithmetic: the products run on the tensor cores.  Each rotated activation group is
+ * scaled by its own power of two (largest magnitude in [2^13, 2^14)) and the codewords by
+ * one power of two per call.  2-bit and ternary codes: both are rounded to 16-bit integers
+ * and multiplied exactly as two int8 planes each (int32 accumulation per group), the group's
+ * four cross products being combined in fp32.  3/4-bit codes: both are rounded to fp16 and
+ * multiplied with fp32 accumulation.  Any finite input is in range; the relative error of y
+ * is about 3e-4 (bound 1e-3 per output vector).  Summation order is fixed: repeated calls
+ * give identical bits.
  *
  *   packed, norms  DEVICE, W quantised as [rows, cols] (rows = outputs, cols = inputs)
  *   rows, cols     >= 0
