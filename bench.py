@@ -99,13 +99,22 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.reader = threading.Thread(target=self._read, daemon=True)
             self.reader.start()
+            # sampling is running before the timed region starts
+            t0 = time.time()
+            while not self.lines and time.time() - t0 < 3.0 and self.proc.poll() is None:
+                time.sleep(0.01)
         except OSError:
             self.proc = None
+        self.first = len(self.lines)
         return self
+
+    def mark(self):
+        """Only samples taken from now on count."""
+        self.first = len(self.lines)
 
     def _read(self):
         for line in self.proc.stdout:
@@ -122,7 +131,7 @@ class ClockSampler:
 
     def summary(self):
         sm, mx, reasons = [], [], set()
-        for ln in self.lines:
+        for ln in self.lines[self.first:]:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) != 6:
                 continue
@@ -401,6 +410,18 @@ def cpu_oracle_sample(target_s: float, threads: int = 0, max_rows: int = 4096):
     return rows * cols * passes / dt / 1e9, rows, passes, dt, nth
 
 
+def arm_config(world: int) -> dict:
+    """The workload both arms report (the reference arm times a bounded sample of it, described
+    in its cpu_baseline.sample)."""
+    from synth import workloads as wlm
+    return {"workload": "llama7b_bf16 weight set (6,476,005,376 weights, 224 tensors), 2-bit "
+                        "quantize_batch + dequantize_batch(bf16) + dequant_gemv_batch (batch 1) over all "
+                        "tensors, per step",
+            "bits": BITS, "group_size": 128, "seed": wlm.LLAMA_7B.seed,
+            "l2": "inputs (12.95 GB) larger than L2; no flush",
+            "parallelism": f"replica per GPU x{world}"}
+
+
 def run_cuda_arm(args):
     import torch
     world, rank, local = dist_env()
@@ -426,6 +447,7 @@ def run_cuda_arm(args):
     barrier()
     torch.cuda.synchronize(device)
     with ClockSampler(nvsmi_id(device)) as clk:
+        clk.mark()
         q_ms, d_ms, g_ms, total_ms = time_phases(ws, args.steps, device)
     torch.cuda.synchronize(device)
     barrier()
@@ -501,11 +523,7 @@ def run_cuda_arm(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": "llama7b_bf16 weight set (6,476,005,376 weights, 224 tensors), "
-                                   "2-bit quantize_batch + dequantize_batch(bf16) + dequant_gemv_batch (batch 1) over all tensors, per step",
-                       "bits": BITS, "group_size": 128, "seed": W.seed,
-                       "l2": "inputs (12.95 GB) larger than L2; no flush",
-                       "parallelism": f"replica per GPU x{world}"},
+            "config": arm_config(world),
             "roofline": {"bound": "hbm", "kernel": f"cq_{dom}", "achieved": round(achieved, 1),
                          "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic},
@@ -610,8 +628,7 @@ def run_reference_arm(args):
         "ms_per_step": round(rows * 4096 * passes / (value * 1e9) * 1e3, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": "llama7b_bf16 weight set, bounded sample (see cpu_baseline.sample)",
-                   "bits": BITS, "group_size": 128, "seed": wlm.LLAMA_7B.seed},
+        "config": arm_config(world),
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": nth, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -664,7 +681,7 @@ def run_ncu_case(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["cq", "reference"], default="cq")
     ap.add_argument("--quick", action="store_true", help="skip the 4-bit and GEMV-replica extras")
