@@ -153,7 +153,11 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     __shared__ __align__(8) uint64_t afull_bar[2], aempty_bar[2], dfull_bar[2], dempty_bar[2];
     __shared__ uint32_t tmem_slot;
     __shared__ uint32_t tab_s[16];  // fp16 (hi | lo << 16) of every code (3- and 4-bit codes)
-    constexpr int kStageBytes = kTile * 16 * B;
+    // norms handed from decode to epilogue, slot i % 4: decode of tile i + 4 waits (through
+    // the MMA of tile i + 2) until the epilogue of tile i has released its D buffer
+    __shared__ float norm_s[4][kTile];
+    constexpr int kCodeBytes = kTile * 16 * B;
+    constexpr int kStageBytes = kCodeBytes + kTile * 2;  // codes, then the tile's fp16 norms
 
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* hmat = smem;
@@ -260,8 +264,12 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                 const long long g0 = (t - jobs.tile0[k]) * kTile;
                 const long long n = sh.total - g0 < kTile ? sh.total - g0 : kTile;
                 const uint32_t bytes = static_cast<uint32_t>(n) * (16 * B);
-                mbar_arrive_expect_tx(&full_bar[st], bytes);
+                // full tiles bring their 256 bytes of norms along (16-byte aligned: the norms
+                // array starts on 16 bytes and a tile's norms start at 256 * tile)
+                const bool nrm_bulk = n == kTile;
+                mbar_arrive_expect_tx(&full_bar[st], bytes + (nrm_bulk ? kTile * 2 : 0));
                 bulk_load(ring + st * kStageBytes, jobs.packed[k] + g0 * (16 * B), bytes, &full_bar[st]);
+                if (nrm_bulk) bulk_load(ring + st * kStageBytes + kCodeBytes, jobs.norms[k] + g0, kTile * 2, &full_bar[st]);
             }
             for (int k = 0; k < kStagesDq && k < i; ++k) {
                 const int ii = i - 1 - k;
@@ -314,6 +322,14 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             const uint32_t a_hi = tbase + lane_off + e * kACols, a_lo = a_hi + 64;
             const long long gid = tl * kTile + m;
             const bool valid = gid < sh.total;
+            {
+                // this group's norm for the epilogue (full tiles: from the stage; the last,
+                // partial tile: from global memory)
+                const bool full_tile = sh.total - tl * kTile >= kTile;
+                const uint16_t* nstage = reinterpret_cast<const uint16_t*>(ring + st * kStageBytes + kCodeBytes);
+                const uint16_t hb = full_tile ? nstage[m] : (valid ? __ldg(jobs.norms[k] + gid) : uint16_t(0));
+                norm_s[i & 3][m] = __half2float(__ushort_as_half(hb));
+            }
             uint32_t wd[4 * B];
             {
                 const uint4* src = reinterpret_cast<const uint4*>(ring + st * kStageBytes + m * (16 * B));
@@ -402,13 +418,12 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             const long long tl = t - jobs.tile0[k];
             const long long gid = tl * kTile + m;
             const bool valid = gid < sh.total;
-            const float nrm = valid ? __half2float(__ushort_as_half(__ldg(jobs.norms[k] + gid))) : 0.0f;
             bool ok = mbar_wait(&dfull_bar[e], (i >> 1) & 1, status);
             // before the staging tile is rewritten, this group's previous stores have read it
             if (sh.flat && leader) bulk_wait_read0();
             if (!named_barrier_and(2 + e, 128, ok)) break;
             tc_fence_after();
-            const float scale = nrm * inv_scale;
+            const float scale = norm_s[i & 3][m] * inv_scale;
             constexpr int kPer = kBF16 ? 8 : 4;  // values per 16-byte chunk
             if (sh.flat) {
                 // stage the tile in shared memory, then one tensor-map store per box
@@ -486,7 +501,7 @@ cudaError_t launch_dq(const DqJobs<NJ>& jobs, const float* cb, unsigned* status,
     // at least 120 KB so that two CTAs never share an SM: each takes all 512 TMEM columns, and
     // with programmatic launch a CTA of the next kernel could otherwise wait inside
     // tcgen05.alloc until the previous one frees them
-    const int smem = std::max(kHBytes + kStagesDq * kTile * 16 * B + 2 * OutTile<kBF16>::kBytes + 1024,
+    const int smem = std::max(kHBytes + kStagesDq * (kTile * 16 * B + kTile * 2) + 2 * OutTile<kBF16>::kBytes + 1024,
                               120 * 1024);
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
