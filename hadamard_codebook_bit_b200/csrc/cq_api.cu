@@ -91,6 +91,16 @@ int resolve_codebook(int bits, const float* codebook, const float** cb) {
 
 }  // namespace
 
+bool is_default_codebook(int bits, const float* cb) {
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices || !bits_ok(bits)) return false;
+    const int slot = slot_for_bits(bits);
+    void* base = nullptr;
+    if (cudaGetSymbolAddress(&base, g_default_codebooks) != cudaSuccess) return false;
+    std::lock_guard<std::mutex> lock(g_mu);
+    return g_default_ready[dev][slot] && cb == static_cast<const float*>(base) + 16 * slot;
+}
+
 unsigned* device_status_ptr() {
     const int dev = current_device();
     if (dev < 0 || dev >= kMaxDevices) return nullptr;

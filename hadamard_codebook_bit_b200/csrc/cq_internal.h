@@ -16,6 +16,8 @@ constexpr int kGroup = 128;
 int levels_for_bits(int bits);
 int field_bits_for(int bits);
 int host_codebook(int bits, int group_size, unsigned long long seed, float* out);
+// True when cb is the default codebook for `bits` on the current device (uploaded already).
+bool is_default_codebook(int bits, const float* cb);
 
 // Number of SMs of the current device (cached per device).
 int sm_count();

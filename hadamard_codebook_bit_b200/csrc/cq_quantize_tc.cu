@@ -28,6 +28,8 @@
 // cols % 128 == 0 the whole matrix is viewed as [groups x 128] (G_eff = 1), so one tile is
 // 128 consecutive groups and the packed output of a tile is one contiguous block.
 #include <algorithm>
+#include <cmath>
+#include <cstring>
 #include <mutex>
 
 #include "cq_device.cuh"
@@ -182,7 +184,9 @@ __device__ __forceinline__ uint32_t bucket_index(float u, const BucketLookup& bl
     return (e & 15u) + (u > __uint_as_float(e) ? 1u : 0u);
 }
 
-template <int B, int L, int NJ>
+// kChecked: the codebook may crowd a bucket, so the kernel checks and keeps the select tree
+// as a fallback; without it (a codebook checked on the host) only the bucket search is built.
+template <int B, int L, int NJ, bool kChecked>
 __global__ void __launch_bounds__(kTcThreads, 1)
     quantize_tc_kernel(const __grid_constant__ TcJobs<NJ> jobs, const float* __restrict__ codebook,
                        unsigned* __restrict__ status) {
@@ -300,7 +304,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int k = 0; k < L - 1; ++k) mid[k] = 0.5f * (__ldg(codebook + k) + __ldg(codebook + k + 1));
         BucketLookup bl{0u, 1.0f, false};
-        if constexpr (B != 2) bl = make_buckets<L>(mid, lane);
+        if constexpr (B != 2) {
+            bl = make_buckets<L>(mid, lane);
+            if constexpr (!kChecked) bl.ok = true;
+        }
         int i = e;
         JobCursor<NJ> cur;
         for (long long t = blockIdx.x + static_cast<long long>(e) * gridDim.x; t < ntiles;
@@ -358,7 +365,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             words[w] |= idx << sh2;
                             if (sh2 + B > 32) words[w + 1] |= idx >> (32 - sh2);
                         }
-                    } else {
+                    } else if constexpr (kChecked) {
 #pragma unroll
                         for (int q = 0; q < 32; ++q) {
                             const uint32_t idx = nearest_index<L>(v[q], T);
@@ -378,7 +385,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                 acc = (acc << B) + bucket_index(v[w * (32 / B) + q] * inv_n, bl);
                             words[B * c + w] = acc;
                         }
-                    } else {
+                    } else if constexpr (kChecked) {
 #pragma unroll
                         for (int w = 0; w < B; ++w) {
                             uint32_t acc = 0u;
@@ -410,7 +417,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
 }
 
-template <int B, int L, int NJ>
+template <int B, int L, int NJ, bool kChecked>
 cudaError_t launch_tc(const TcJobs<NJ>& jobs, const float* cb, unsigned* status, cudaStream_t st) {
     const int smem = (1 + kStagesTc) * kTileBytes + 1024;
     int dev = 0;
@@ -419,13 +426,13 @@ cudaError_t launch_tc(const TcJobs<NJ>& jobs, const float* cb, unsigned* status,
     static unsigned long long configured = 0;
     const unsigned long long bit = 1ull << (dev & 63);
     if (!(configured & bit)) {
-        e = cudaFuncSetAttribute(quantize_tc_kernel<B, L, NJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        e = cudaFuncSetAttribute(quantize_tc_kernel<B, L, NJ, kChecked>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         configured |= bit;
     }
     const long long ntiles = jobs.tile0[jobs.n];
     const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(ntiles, sm_count())));
-    return launch_pdl(quantize_tc_kernel<B, L, NJ>, dim3(grid), dim3(kTcThreads), smem, st, jobs, cb, status);
+    return launch_pdl(quantize_tc_kernel<B, L, NJ, kChecked>, dim3(grid), dim3(kTcThreads), smem, st, jobs, cb, status);
 }
 
 // Shape, tensor map and outputs of one tensor as job k of `jobs`.
@@ -454,13 +461,51 @@ bool add_job(TcJobs<NJ>& jobs, int k, const void* w, const Shape& sh, uint8_t* p
     return true;
 }
 
+// The bucket table of make_buckets built on the host with the same fp32 operations: true when
+// no bucket receives two midpoints of codebook c (L levels).
+bool buckets_ok_host(const float* c, int L) {
+    float mid[15];
+    for (int k = 0; k < L - 1; ++k) mid[k] = 0.5f * (c[k] + c[k + 1]);
+    float span = std::max(std::fabs(mid[0]), std::fabs(mid[L - 2])) * 1.1f;
+    if (!(span > 0.0f)) span = 1.0f;
+    const float sA = 0.5f / span;
+    int cnt[32] = {0};
+    for (int k = 0; k < L - 1; ++k) {
+        float tt = std::fmaf(mid[k], sA, 0.5f);
+        tt = tt > 0.0f ? (tt < 1.0f ? tt : 1.0f) : 0.0f;  // saturate (NaN -> 0)
+        const float q = std::fmaf(tt, 31.0f, 12582912.0f);
+        uint32_t bits = 0;
+        std::memcpy(&bits, &q, sizeof(bits));
+        if (++cnt[bits & 31u] > 1) return false;
+    }
+    return true;
+}
+
+// True when cb is this library's default codebook for `bits` and its bucket table is clean
+// (then the kernel needs no in-kernel check and no select-tree fallback).
+bool default_codebook_is_clean(int bits, const float* cb) {
+    if (bits != 3 && bits != 4) return false;
+    if (!is_default_codebook(bits, cb)) return false;
+    static int clean[5] = {-1, -1, -1, -1, -1};  // per bits; the default codebooks never change
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    if (clean[bits] < 0) {
+        float host[16] = {0};
+        clean[bits] = (host_codebook(bits, kTile, 0, host) == (1 << bits) && buckets_ok_host(host, 1 << bits)) ? 1 : 0;
+    }
+    return clean[bits] == 1;
+}
+
 template <int NJ>
 cudaError_t launch_bits(int bits, const TcJobs<NJ>& jobs, const float* cb, unsigned* status, cudaStream_t st) {
+    const bool clean = default_codebook_is_clean(bits, cb);
     switch (bits) {
-        case CQ_BITS_TERNARY: return launch_tc<2, 3, NJ>(jobs, cb, status, st);
-        case 2: return launch_tc<2, 4, NJ>(jobs, cb, status, st);
-        case 3: return launch_tc<3, 8, NJ>(jobs, cb, status, st);
-        default: return launch_tc<4, 16, NJ>(jobs, cb, status, st);
+        case CQ_BITS_TERNARY: return launch_tc<2, 3, NJ, false>(jobs, cb, status, st);
+        case 2: return launch_tc<2, 4, NJ, false>(jobs, cb, status, st);
+        case 3:
+            return clean ? launch_tc<3, 8, NJ, false>(jobs, cb, status, st) : launch_tc<3, 8, NJ, true>(jobs, cb, status, st);
+        default:
+            return clean ? launch_tc<4, 16, NJ, false>(jobs, cb, status, st) : launch_tc<4, 16, NJ, true>(jobs, cb, status, st);
     }
 }
 
