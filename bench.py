@@ -682,7 +682,7 @@ def run_ncu_case(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["cq", "reference"], default="cq")
     ap.add_argument("--quick", action="store_true", help="skip the 4-bit and GEMV-replica extras")
