@@ -30,7 +30,7 @@ _STATUS = {0: "CQ_OK", 1: "CQ_ERR_INVALID_ARG", 2: "CQ_ERR_UNSUPPORTED", 3: "CQ_
 EXPORTS = ("cq_status_string", "cq_version", "cq_device_status", "cq_codebook", "cq_packed_bytes",
            "cq_norm_bytes", "cq_quantize", "cq_dequantize", "cq_dequant_gemv",
            "cq_gemv_workspace_bytes", "cq_dequant_gemv_static", "cq_quantize_batch",
-           "cq_dequantize_batch", "cq_dequant_gemv_batch")
+           "cq_dequantize_batch", "cq_dequant_gemv_batch", "cq_fake_quantize", "cq_fake_quantize_batch")
 
 
 class CQError(RuntimeError):
@@ -69,6 +69,8 @@ def lib() -> ctypes.CDLL:
         L.cq_quantize_batch.argtypes = [P, i, i, i, i, P, P]
         L.cq_dequantize_batch.argtypes = [P, i, i, i, P, i, P]
         L.cq_dequant_gemv_batch.argtypes = [P, i, i, i, P, P]
+        L.cq_fake_quantize.argtypes = [P, i, ll, ll, i, i, P, P, P, P, i, P]
+        L.cq_fake_quantize_batch.argtypes = [P, i, i, i, i, P, i, P]
         _lib = L
     return _lib
 
@@ -282,6 +284,75 @@ def dequant_gemv_batch(items, bits: int, group_size: int = GROUP_SIZE, codebook=
                                            group_size, _cb_ptr(codebook, dev), _stream(dev)),
                "cq_dequant_gemv_batch")
     return out
+
+
+def _dtype_code(dtype, what: str) -> int:
+    torch = _torch()
+    if dtype == torch.bfloat16:
+        return CQ_BF16
+    if dtype == torch.float32:
+        return CQ_F32
+    raise ValueError(f"{what} must be bfloat16 or float32")
+
+
+def fake_quantize(w, bits: int, group_size: int = GROUP_SIZE, codebook=None, out_dtype=None,
+                  out=None, stored=None):
+    """cq_fake_quantize -> W_hat = dequantize(quantize(w)), the tensor the pages' cq_quantize
+    returns (same dtype as w unless `out_dtype` / `out` say otherwise; `out=w` works in place).
+    `stored`, if given, is the (packed, norms) pair that receives the stored form."""
+    torch = _torch()
+    if w.dim() != 2:
+        raise ValueError("w must be 2-D [rows, cols]")
+    wt = _dtype_code(w.dtype, "w")
+    rows, cols = w.shape
+    if out is None:
+        out = torch.empty((rows, cols), dtype=w.dtype if out_dtype is None else out_dtype, device=w.device)
+    ot = _dtype_code(out.dtype, "out")
+    packed, norms = stored if stored is not None else empty_packed(rows, cols, bits, w.device, group_size)
+    with torch.cuda.device(w.device):
+        _check(lib().cq_fake_quantize(_dev_ptr(w, "w"), wt, rows, cols, bits, group_size,
+                                      _cb_ptr(codebook, w.device), _dev_ptr(packed, "packed"),
+                                      _dev_ptr(norms, "norms"), _dev_ptr(out, "out"), ot,
+                                      _stream(w.device)), "cq_fake_quantize")
+    return out
+
+
+class _FakeQuantizeJob(ctypes.Structure):  # cq_fake_quantize_job
+    _fields_ = [("w", ctypes.c_void_p), ("rows", ctypes.c_longlong), ("cols", ctypes.c_longlong),
+                ("packed_out", ctypes.c_void_p), ("norms_out", ctypes.c_void_p), ("out", ctypes.c_void_p)]
+
+
+def fake_quantize_batch(ws, bits: int, group_size: int = GROUP_SIZE, codebook=None, out_dtype=None,
+                        outs=None, stored=None):
+    """cq_fake_quantize_batch on a list of 2-D CUDA tensors of one dtype on one device ->
+    list of W_hat tensors (`outs` may be `ws` itself for in-place fake quantisation).
+    `stored`, if given, is a list of (packed, norms) pairs receiving the stored forms."""
+    torch = _torch()
+    if not ws:
+        return []
+    dev = ws[0].device
+    wt = _dtype_code(ws[0].dtype, "w")
+    if outs is None:
+        odt = ws[0].dtype if out_dtype is None else out_dtype
+        outs = [torch.empty(tuple(w.shape), dtype=odt, device=dev) for w in ws]
+    ot = _dtype_code(outs[0].dtype, "out")
+    jobs = (_FakeQuantizeJob * len(ws))()
+    keep = []  # intermediate buffers stay allocated until the launches are enqueued
+    for k, (w, out) in enumerate(zip(ws, outs)):
+        if w.dim() != 2 or w.dtype != ws[0].dtype or w.device != dev:
+            raise ValueError("tensors must be 2-D, of one dtype, on one device")
+        if out.dtype != outs[0].dtype or out.device != dev or tuple(out.shape) != tuple(w.shape):
+            raise ValueError("outputs must match their inputs' shapes and share one dtype")
+        rows, cols = w.shape
+        packed, norms = stored[k] if stored is not None else empty_packed(rows, cols, bits, dev, group_size)
+        keep.append((packed, norms))
+        jobs[k] = _FakeQuantizeJob(_dev_ptr(w, "w"), rows, cols, _dev_ptr(packed, "packed"),
+                                   _dev_ptr(norms, "norms"), _dev_ptr(out, "out"))
+    with torch.cuda.device(dev):
+        _check(lib().cq_fake_quantize_batch(ctypes.cast(jobs, ctypes.c_void_p), len(ws), wt, bits,
+                                            group_size, _cb_ptr(codebook, dev), ot, _stream(dev)),
+               "cq_fake_quantize_batch")
+    return outs
 
 
 def dequantize(packed, norms, rows: int, cols: int, bits: int, group_size: int = GROUP_SIZE,

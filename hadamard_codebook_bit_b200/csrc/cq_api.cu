@@ -2,6 +2,7 @@
 //
 // Host side only: argument validation (before any launch), the per-device default
 // codebook, and dispatch to the kernel launchers.  Nothing here computes on the data.
+#include <algorithm>
 #include <cstdint>
 #include <cstdlib>
 #include <mutex>
@@ -87,6 +88,24 @@ int resolve_codebook(int bits, const float* codebook, const float** cb) {
         return CQ_OK;
     }
     return default_codebook(bits, cb) == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
+}
+
+// Activation rows per GEMV launch job (the tensor-core B operand holds 8 batch columns).
+// Larger batches, up to kMaxGemvBatch, become ceil(batch / 8) jobs of the same launch pair,
+// one per block of 8 rows of x and y, each with its own slice of the caller's workspace.
+constexpr int kGemvChunk = 8;
+constexpr int kMaxGemvBatch = 64;
+
+void push_gemv_chunks(std::vector<GemvItem>& items, const unsigned char* packed,
+                      const unsigned short* norms, long long rows, long long cols, const void* x,
+                      int batch, float* y, void* workspace) {
+    const size_t chunk_ws = gemv_workspace_bytes(cols, kGemvChunk);
+    const Shape sh = make_shape(rows, cols);
+    for (int c0 = 0; c0 < batch; c0 += kGemvChunk) {
+        items.push_back({packed, norms, sh, static_cast<const uint16_t*>(x) + static_cast<long long>(c0) * cols,
+                         std::min(kGemvChunk, batch - c0), y + static_cast<long long>(c0) * rows,
+                         static_cast<char*>(workspace) + static_cast<size_t>(c0 / kGemvChunk) * chunk_ws});
+    }
 }
 
 }  // namespace
@@ -321,13 +340,59 @@ int cq_dequantize_batch(const cq_dequantize_job* jobs, int count, int bits, int 
     return CQ_OK;
 }
 
+int cq_fake_quantize(const void* w, int w_dtype, long long rows, long long cols, int bits,
+                     int group_size, const float* codebook, unsigned char* packed_out,
+                     unsigned short* norms_out, void* out, int out_dtype, void* stream) {
+    // Validate what the dequantise step adds before the quantise step launches anything.
+    if (out_dtype != CQ_F32 && out_dtype != CQ_BF16) return CQ_ERR_INVALID_ARG;
+    if (w_dtype != CQ_F32 && w_dtype != CQ_BF16) return CQ_ERR_INVALID_ARG;
+    const int rc = cq::check_common(rows, cols, bits, group_size);
+    if (rc != CQ_OK) return rc;
+    if (rows == 0 || cols == 0) return CQ_OK;
+    if (!out) return CQ_ERR_INVALID_ARG;
+    if (!cq::aligned16(out)) return CQ_ERR_ALIGNMENT;
+    const cq_fake_quantize_job job = {w, rows, cols, packed_out, norms_out, out};
+    return cq_fake_quantize_batch(&job, 1, w_dtype, bits, group_size, codebook, out_dtype, stream);
+}
+
+int cq_fake_quantize_batch(const cq_fake_quantize_job* jobs, int count, int w_dtype, int bits,
+                           int group_size, const float* codebook, int out_dtype, void* stream) {
+    if (count < 0 || (count > 0 && !jobs)) return CQ_ERR_INVALID_ARG;
+    if (w_dtype != CQ_F32 && w_dtype != CQ_BF16) return CQ_ERR_INVALID_ARG;
+    if (out_dtype != CQ_F32 && out_dtype != CQ_BF16) return CQ_ERR_INVALID_ARG;
+    std::vector<cq_quantize_job> q;
+    std::vector<cq_dequantize_job> d;
+    q.reserve(static_cast<size_t>(count));
+    d.reserve(static_cast<size_t>(count));
+    for (int i = 0; i < count; ++i) {
+        const cq_fake_quantize_job& j = jobs[i];
+        const int rc = cq::check_common(j.rows, j.cols, bits, group_size);
+        if (rc != CQ_OK) return rc;
+        if (j.rows == 0 || j.cols == 0) continue;
+        if (!j.w || !j.packed_out || !j.norms_out || !j.out) return CQ_ERR_INVALID_ARG;
+        if (!cq::aligned16(j.w) || !cq::aligned16(j.packed_out) || !cq::aligned16(j.norms_out) ||
+            !cq::aligned16(j.out))
+            return CQ_ERR_ALIGNMENT;
+        q.push_back({j.w, j.rows, j.cols, j.packed_out, j.norms_out});
+        d.push_back({j.packed_out, j.norms_out, j.rows, j.cols, j.out});
+    }
+    if (q.empty()) return CQ_OK;
+    if (codebook != nullptr && (reinterpret_cast<uintptr_t>(codebook) & 3u) != 0) return CQ_ERR_ALIGNMENT;
+    // Both steps now pass their own validation; only a CUDA failure can stop the second.
+    const int rc = cq_quantize_batch(q.data(), static_cast<int>(q.size()), w_dtype, bits, group_size,
+                                     codebook, stream);
+    if (rc != CQ_OK) return rc;
+    return cq_dequantize_batch(d.data(), static_cast<int>(d.size()), bits, group_size, codebook,
+                               out_dtype, stream);
+}
+
 int cq_dequant_gemv_batch(const cq_gemv_job* jobs, int count, int bits, int group_size,
                           const float* codebook, void* stream) {
     if (count < 0 || (count > 0 && !jobs)) return CQ_ERR_INVALID_ARG;
     bool any = false;
     for (int i = 0; i < count; ++i) {
         const cq_gemv_job& j = jobs[i];
-        if (j.batch < 1 || j.batch > 8) return CQ_ERR_INVALID_ARG;
+        if (j.batch < 1 || j.batch > cq::kMaxGemvBatch) return CQ_ERR_INVALID_ARG;
         const int rc = cq::check_common(j.rows, j.cols, bits, group_size);
         if (rc != CQ_OK) return rc;
         if (j.rows == 0) continue;
@@ -354,8 +419,7 @@ int cq_dequant_gemv_batch(const cq_gemv_job* jobs, int count, int bits, int grou
             if (e != cudaSuccess) return CQ_ERR_CUDA;
             continue;
         }
-        items.push_back({j.packed, j.norms, cq::make_shape(j.rows, j.cols),
-                         static_cast<const uint16_t*>(j.x), j.batch, j.y, j.workspace});
+        cq::push_gemv_chunks(items, j.packed, j.norms, j.rows, j.cols, j.x, j.batch, j.y, j.workspace);
     }
     if (items.empty()) return CQ_OK;
     const float* cb = nullptr;
@@ -366,7 +430,7 @@ int cq_dequant_gemv_batch(const cq_gemv_job* jobs, int count, int bits, int grou
 }
 
 size_t cq_gemv_workspace_bytes(long long cols, int batch) {
-    if (cols < 0 || batch < 1 || batch > 8) return 0;
+    if (cols < 0 || batch < 1 || batch > cq::kMaxGemvBatch) return 0;
     return cq::gemv_workspace_bytes(cols, batch);
 }
 
@@ -374,7 +438,7 @@ int cq_dequant_gemv(const unsigned char* packed, const unsigned short* norms, lo
                     long long cols, int bits, int group_size, const float* codebook,
                     const void* x, int batch, float* y, void* workspace,
                     size_t workspace_bytes, void* stream) {
-    if (batch < 1 || batch > 8) return CQ_ERR_INVALID_ARG;
+    if (batch < 1 || batch > cq::kMaxGemvBatch) return CQ_ERR_INVALID_ARG;
     int rc = cq::check_common(rows, cols, bits, group_size);
     if (rc != CQ_OK) return rc;
     if (rows == 0) return CQ_OK;  // y is empty
@@ -395,9 +459,16 @@ int cq_dequant_gemv(const unsigned char* packed, const unsigned short* norms, lo
     const float* cb = nullptr;
     rc = cq::resolve_codebook(bits, codebook, &cb);
     if (rc != CQ_OK) return rc;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (batch > cq::kGemvChunk) {  // one launch pair over the blocks of 8 activation rows
+        std::vector<cq::GemvItem> items;
+        cq::push_gemv_chunks(items, packed, norms, rows, cols, x, batch, y, workspace);
+        const cudaError_t e = cq::launch_dequant_gemv_batch(items.data(), static_cast<int>(items.size()), bits, cb, st);
+        return e == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
+    }
     const cudaError_t e = cq::launch_dequant_gemv(
         packed, norms, cq::make_shape(rows, cols), bits, cb, static_cast<const uint16_t*>(x),
-        batch, y, workspace, static_cast<cudaStream_t>(stream));
+        batch, y, workspace, st);
     return e == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
 }
 

@@ -765,10 +765,11 @@ static_assert(sizeof(GemvJobs<kGemvBatch>) < 32000, "kernel parameter space");
 }  // namespace
 
 size_t gemv_workspace_bytes(long long cols, int batch) {
-    (void)batch;  // the B operand is always padded to 8 columns
+    // one block per 8 activation rows (the B operand is always padded to 8 columns)
     const long long G = (cols + kGroup - 1) / kGroup;
     const size_t bytes = frag_bytes(G) + scale_bytes(G) + sizeof(CodeTable);
-    return (bytes + 255) / 256 * 256;
+    const size_t blocks = static_cast<size_t>(batch < 1 ? 1 : (batch + kBatchCols - 1) / kBatchCols);
+    return (bytes + 255) / 256 * 256 * blocks;
 }
 
 cudaError_t launch_dequant_gemv(const uint8_t* packed, const uint16_t* norms, const Shape& sh,

@@ -211,6 +211,54 @@ int cq_dequantize_batch(const cq_dequantize_job* jobs, int count, int bits, int 
                         const float* codebook, int out_dtype, void* stream);
 
 /*
+ * cq_fake_quantize -- W_hat = dequantize(quantize(W)) in one call: the tensor that the
+ * pages' cq_quantize returns.
+ *
+ * Page "Cactus Quants CQ2-bit Quantization", "The CQ2-bit Implementation Pipeline" steps
+ * 1-6 (pad, rotate, normalise, nearest codeword, inverse rotate, unpad), whose output is the
+ * de-quantised tensor; page "How Quantization Codebooks Are Trained in Cactus Quants",
+ * "Practical Usage Example" (cq_quantize applied with a caller codebook).  The scale
+ * used for the inverse rotation is the stored fp16 norm, so W_hat is bit for bit what
+ * cq_dequantize reconstructs from the stored form that cq_quantize writes.
+ *
+ *   w, w_dtype, rows, cols, bits, group_size, codebook   as for cq_quantize
+ *   packed_out, norms_out   DEVICE buffers as for cq_quantize; they receive the stored form
+ *                           (the intermediate; the caller may discard it)
+ *   out, out_dtype          as for cq_dequantize.  out may be w itself (in-place fake
+ *                           quantisation, when the dtypes match): every read of w completes
+ *                           before the first write of out.  It must not overlap packed_out
+ *                           or norms_out.
+ * Two launches on `stream` (quantise, then dequantise).  Every argument is validated before
+ * anything is launched.  Returns CQ_OK after enqueueing, or an error with nothing launched.
+ */
+int cq_fake_quantize(const void* w, int w_dtype, long long rows, long long cols, int bits,
+                     int group_size, const float* codebook, unsigned char* packed_out,
+                     unsigned short* norms_out, void* out, int out_dtype, void* stream);
+
+/*
+ * cq_fake_quantize_batch -- cq_fake_quantize over a list of tensors: one cq_quantize_batch
+ * over all jobs, then one cq_dequantize_batch.  Every w is read before any out is written,
+ * so outputs may alias any job's w; otherwise the rules of the two batched calls apply (no
+ * job's packed_out / norms_out may overlap another job's buffers or any out).
+ *
+ *   jobs        HOST array of `count` descriptors, read during the call only
+ *   count       >= 0 (0: nothing to do)
+ * Every job is validated before anything is launched; the first failing job's status is
+ * returned.  Returns CQ_OK after enqueueing.
+ */
+typedef struct cq_fake_quantize_job {
+    const void* w;
+    long long rows;
+    long long cols;
+    unsigned char* packed_out;
+    unsigned short* norms_out;
+    void* out;
+} cq_fake_quantize_job;
+
+int cq_fake_quantize_batch(const cq_fake_quantize_job* jobs, int count, int w_dtype, int bits,
+                           int group_size, const float* codebook, int out_dtype, void* stream);
+
+/*
  * cq_dequant_gemv -- y = W_hat x without materialising W_hat.
  *
  * Because H is symmetric and orthonormal (page "How CQ2-bit Quantization Contributes to
@@ -235,12 +283,16 @@ int cq_dequantize_batch(const cq_dequantize_job* jobs, int count, int bits, int 
  *   group_size     must be 128
  *   codebook       DEVICE L fp32 ascending, or NULL for the default
  *   x              DEVICE bf16 [batch, cols], row-major
- *   batch          1..8
+ *   batch          1..64.  The tensor cores take 8 activation rows at a time: a batch above 8
+ *                  runs as ceil(batch / 8) blocks of at most 8 rows in the same launches,
+ *                  each block streaming the packed weights again (from L2 while they stay
+ *                  resident), so HBM traffic for the weights grows with ceil(batch / 8).
  *   y              DEVICE fp32 [batch, rows], row-major, overwritten
  *   workspace      DEVICE scratch of at least cq_gemv_workspace_bytes(cols, batch) bytes
- *                  (2080 bytes per 128 columns plus 48), 16-byte aligned; its contents on entry are
- *                  ignored and on return are unspecified.  Calls that overlap in time must
- *                  not share a workspace.
+ *                  (2080 bytes per 128 columns plus 48, rounded up to 256, per block of 8
+ *                  activation rows), 16-byte aligned; its contents on entry are ignored and
+ *                  on return are unspecified.  Calls that overlap in time must not share a
+ *                  workspace.
  */
 int cq_dequant_gemv(const unsigned char* packed, const unsigned short* norms, long long rows,
                     long long cols, int bits, int group_size, const float* codebook,
@@ -291,6 +343,8 @@ size_t cq_gemv_workspace_bytes(long long cols, int batch);
  * routine.  Same arguments, semantics and results as cq_dequant_gemv, minus the workspace.
  *
  *   cols       at most 32768; larger returns CQ_ERR_WORKSPACE and launches nothing
+ *   batch      1..64; the array holds one block of 8 activation rows, so a batch above 8
+ *              runs as consecutive launch pairs on `stream`, one per block
  *   set-up     the first call on each device looks up the array's device address (a
  *              synchronous runtime call); make that first call before any stream capture
  *   sharing    every call on a device uses the same array, which keeps the last call's

@@ -213,6 +213,18 @@ def dequantize(packed: np.ndarray, norms: np.ndarray, rows: int, cols: int, bits
     return out
 
 
+def fake_quantize(w: np.ndarray, bits: int, group_size: int = 128,
+                  codebook_: np.ndarray | None = None, nthreads: int = 0) -> np.ndarray:
+    """W_hat [rows, cols] fp64 = dequantize(quantize(w)): the de-quantised tensor the pages'
+    cq_quantize returns (page "Cactus Quants CQ2-bit Quantization", "The CQ2-bit
+    Implementation Pipeline", steps 1-6).  The inverse rotation scales by the stored fp16
+    norm, so the result is what a deployment reconstructs from the stored form."""
+    w = np.ascontiguousarray(w)
+    rows, cols = w.shape
+    packed, norms = quantize(w, bits, group_size, codebook_, nthreads=nthreads)
+    return dequantize(packed, norms, rows, cols, bits, group_size, codebook_, nthreads)
+
+
 def dequant_gemv(packed: np.ndarray, norms: np.ndarray, rows: int, cols: int, bits: int,
                  x: np.ndarray, group_size: int = 128, codebook_: np.ndarray | None = None,
                  nthreads: int = 0) -> np.ndarray:

@@ -200,6 +200,26 @@ def test_gemv_all_bits_and_ragged(ora, bits, cols, batch):
     parity.check_gemv(to_np(y), y_ref, f"gemv bits={bits} cols={cols}")
 
 
+@pytest.mark.parametrize("bits", [0, 2, 3, 4])
+@pytest.mark.parametrize("batch", [9, 16, 33, 64])
+def test_gemv_prefill_batches(ora, bits, batch):
+    """Batches above 8 activation rows (up to 64) run as blocks of 8 in one launch pair."""
+    rows, cols = 70, 1000
+    w_dev = dev_tensor(rows, cols, torch.bfloat16, 15, batch + bits, 0.02)
+    packed, norms = cq.quantize(w_dev, bits)
+    x = torch.empty((batch, cols), dtype=torch.bfloat16, device=DEV)
+    synth.fill_normal_(x, 15, 2000 + batch, 1.0)
+    y = cq.dequant_gemv(packed, norms, rows, cols, bits, x)
+    y_ref = ora.dequant_gemv(to_np(packed), to_np(norms), rows, cols, bits, to_np(x))
+    parity.check_gemv(to_np(y), y_ref, f"gemv bits={bits} batch={batch}")
+    # the batched entry point with mixed batch sizes gives the same products
+    x8 = x[:8].contiguous()
+    ys = cq.dequant_gemv_batch([(packed, norms, rows, cols, x), (packed, norms, rows, cols, x8)], bits)
+    torch.cuda.synchronize()
+    parity.check_gemv(to_np(ys[0]), y_ref, f"gemv batch-call bits={bits} batch={batch}")
+    parity.check_gemv(to_np(ys[1]), y_ref[:8], f"gemv batch-call bits={bits} batch=8")
+
+
 def test_zero_and_spike_groups(ora):
     w = torch.zeros((6, 384), dtype=torch.float32, device=DEV)
     w[1, 5] = 0.37
@@ -351,6 +371,86 @@ def test_dequantize_batch_many_jobs():
     got = cq.dequantize_batch(items, 2)
     for (pk, nm, r, c), ob in zip(items, got):
         assert torch.equal(ob.view(torch.int16), cq.dequantize(pk, nm, r, c, 2).view(torch.int16))
+
+
+# ------------------------------------------------------------------------------------------
+# fake quantisation: W_hat = dequantize(quantize(W)) in one call
+# ------------------------------------------------------------------------------------------
+
+def _int_view(t):
+    return t.view(torch.int16) if t.element_size() == 2 else t.view(torch.int32)
+
+
+def fake_check(ora, w_dev, bits, out_dtype, what):
+    """cq_fake_quantize against (1) the library's own two-step result, bit for bit, and
+    (2) the oracle's fake quantisation of the same input, group by group where the stored
+    forms agree, and the oracle's dequantisation of the GPU's stored form where an index sits
+    inside the boundary band (check_indices bounds those)."""
+    rows, cols = w_dev.shape
+    stored = cq.empty_packed(rows, cols, bits, w_dev.device)
+    out = cq.fake_quantize(w_dev, bits, out_dtype=out_dtype, stored=stored)
+    ps, ns = cq.quantize(w_dev, bits)
+    assert torch.equal(stored[0], ps) and torch.equal(stored[1].view(torch.int16), ns.view(torch.int16))
+    two_step = cq.dequantize(ps, ns, rows, cols, bits, out_dtype=out_dtype)
+    assert out.dtype == out_dtype and torch.equal(_int_view(out), _int_view(two_step))
+    w_np = to_np(w_dev)
+    o_packed, o_norms, u = ora.quantize(w_np, bits, want_u=True)
+    g_packed, g_norms = to_np(ps), to_np(ns)
+    parity.check_indices(g_packed, o_packed, u, bits, cq.codebook(bits), what)
+    w64 = w_np.astype(np.float64) if w_np.dtype != np.uint16 else parity.bf16_to_f64(w_np).reshape(rows, cols)
+    parity.check_norms(g_norms, o_norms, parity.group_norms(w64, cols), what)
+    ref = ora.fake_quantize(w_np, bits)
+    same = np.all(g_packed == o_packed, axis=-1) & (g_norms == o_norms)  # [rows, G]
+    if not same.all():
+        alt = ora.dequantize(g_packed, g_norms, rows, cols, bits)
+        cmask = np.repeat(same, 128, axis=1)[:, :cols]
+        ref = np.where(cmask, ref, alt)
+    if out_dtype == torch.float32:
+        parity.check_dequant_f32(to_np(out), ref, cols, what)
+    else:
+        parity.check_dequant_bf16(to_np(out), ref, cols, what)
+    return int((~same).sum())
+
+
+@pytest.mark.parametrize("bits", [0, 2, 3, 4])
+@pytest.mark.parametrize("cols", [128, 1000, 4096])
+def test_fake_quantize_matches_oracle(ora, bits, cols):
+    w_dev = dev_tensor(70, cols, torch.bfloat16, 40, cols + bits, 0.02)
+    fake_check(ora, w_dev, bits, torch.bfloat16, f"fake bf16 bits={bits} cols={cols}")
+    fake_check(ora, w_dev, bits, torch.float32, f"fake bf16->f32 bits={bits} cols={cols}")
+
+
+@pytest.mark.parametrize("cols", [1, 129, 4100])
+def test_fake_quantize_fp32_ragged_and_special(ora, cols):
+    w_dev = dev_tensor(33, cols, torch.float32, 41, cols, 1.0)
+    w_dev[3, :] = 0.0
+    w_dev[4, :] = 0.0
+    w_dev[4, cols // 2] = -2.5  # spike group
+    for bits in (0, 2, 4):
+        fake_check(ora, w_dev, bits, torch.float32, f"fake f32 bits={bits} cols={cols}")
+
+
+def test_fake_quantize_in_place_and_batch():
+    """out = w (in place) gives the out-of-place result; the batched call gives the single
+    calls' bytes, in place too, over assorted (and empty) shapes."""
+    w = dev_tensor(300, 4096, torch.bfloat16, 42, 0, 0.02)
+    want = cq.fake_quantize(w, 2)
+    w2 = w.clone()
+    got = cq.fake_quantize(w2, 2, out=w2)
+    assert got.data_ptr() == w2.data_ptr() and torch.equal(_int_view(w2), _int_view(want))
+    ws = [batch_tensor(r, c, torch.bfloat16, 43, k, 0.02) for k, (r, c) in enumerate(BATCH_SHAPES)]
+    singles = [cq.fake_quantize(x, 4) for x in ws]
+    outs = cq.fake_quantize_batch(ws, 4)
+    for a, b in zip(outs, singles):
+        assert a.shape == b.shape and torch.equal(_int_view(a), _int_view(b))
+    copies = [x.clone() for x in ws]
+    cq.fake_quantize_batch(copies, 4, outs=copies)
+    for a, b in zip(copies, singles):
+        assert torch.equal(_int_view(a), _int_view(b))
+    many = [dev_tensor(2 + k % 5, 128 * (1 + k % 3), torch.float32, 44, k, 1.0) for k in range(150)]
+    outs = cq.fake_quantize_batch(many, 3, out_dtype=torch.bfloat16)
+    for k in (0, 127, 128, 149):
+        assert torch.equal(_int_view(outs[k]), _int_view(cq.fake_quantize(many[k], 3, out_dtype=torch.bfloat16)))
 
 
 @pytest.mark.parametrize("bits", [0, 2, 4])

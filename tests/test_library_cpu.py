@@ -87,7 +87,9 @@ def test_byte_counts_edge_cases(L):
     assert cq.gemv_workspace_bytes(4096, 1) == ws(32) == cq.gemv_workspace_bytes(4096, 8)
     assert cq.gemv_workspace_bytes(11008, 8) == ws(86)
     assert cq.gemv_workspace_bytes(1, 3) == ws(1)
-    assert cq.gemv_workspace_bytes(4096, 9) == 0 and cq.gemv_workspace_bytes(4096, 0) == 0
+    assert cq.gemv_workspace_bytes(4096, 9) == 2 * ws(32) == cq.gemv_workspace_bytes(4096, 16)
+    assert cq.gemv_workspace_bytes(4096, 64) == 8 * ws(32)
+    assert cq.gemv_workspace_bytes(4096, 65) == 0 and cq.gemv_workspace_bytes(4096, 0) == 0
 
 
 # ------------------------------------------------------------------------------------------
@@ -132,7 +134,11 @@ def test_gemv_rejects(L):
     g = L.cq_dequant_gemv
     ws = cq.gemv_workspace_bytes(256, 1)
     assert g(A, A, 4, 256, 2, 128, None, A, 0, A, A, ws, None) == 1    # batch 0
-    assert g(A, A, 4, 256, 2, 128, None, A, 9, A, A, ws, None) == 1    # batch 9
+    assert g(A, A, 4, 256, 2, 128, None, A, 65, A, A, ws, None) == 1   # batch 65
+    ws64 = cq.gemv_workspace_bytes(256, 64)
+    assert ws64 == 8 * cq.gemv_workspace_bytes(256, 8) and cq.gemv_workspace_bytes(256, 9) == 2 * ws
+    assert g(A, A, 4, 256, 2, 128, None, A, 9, A, A, ws, None) == 5    # batch 9 needs two blocks
+    assert g(A, A, 4, 256, 2, 128, None, A, 64, A, A, ws64 - 1, None) == 5
     assert g(A, A, 4, 256, 2, 128, None, None, 1, A, A, ws, None) == 1  # null x
     assert g(A, A, 4, 256, 2, 128, None, A, 1, A, None, ws, None) == 5  # no workspace
     assert g(A, A, 4, 256, 2, 128, None, A, 1, A, A, ws - 1, None) == 5
@@ -205,14 +211,51 @@ def test_gemv_batch_rejects_before_launching(L):
     assert g(p, -1, 2, 128, None, None) == 1
     assert g(None, 2, 2, 128, None, None) == 1
     assert g(p, 2, 5, 128, None, None) == 1                          # bits 5
+    p, _k = jobs(good, (A, A, 4, 256, A, 65, A, A, 8 * ws))
+    assert g(p, 2, 2, 128, None, None) == 1                          # batch 65
     p, _k = jobs(good, (A, A, 4, 256, A, 9, A, A, ws))
-    assert g(p, 2, 2, 128, None, None) == 1                          # batch 9
+    assert g(p, 2, 2, 128, None, None) == 5                          # batch 9: two blocks of workspace
     p, _k = jobs(good, (A, A, 4, 256, A, 1, A, A, ws - 1))
     assert g(p, 2, 2, 128, None, None) == 5                          # workspace too small
     p, _k = jobs(good, (A, A, 4, 256, A, 1, A + 4, A, ws))
     assert g(p, 2, 2, 128, None, None) == 4                          # misaligned y
     p, _k = jobs((None, None, 0, 256, None, 1, None, None, 0))
     assert g(p, 1, 2, 128, None, None) == 0                          # rows == 0: nothing to do
+
+
+def _fjobs(*jobs):
+    arr = (cq._FakeQuantizeJob * max(1, len(jobs)))()
+    for k, j in enumerate(jobs):
+        arr[k] = cq._FakeQuantizeJob(*j)
+    return ctypes.cast(arr, ctypes.c_void_p), arr
+
+
+def test_fake_quantize_rejects_before_launching(L):
+    f = L.cq_fake_quantize
+    assert f(A, 2, 4, 128, 2, 128, None, A, A, A, 1, None) == 1       # bad w dtype
+    assert f(A, 1, 4, 128, 2, 128, None, A, A, A, 2, None) == 1       # bad out dtype
+    assert f(A, 1, 4, 128, 5, 128, None, A, A, A, 1, None) == 1       # bits 5
+    assert f(A, 1, 4, 128, 2, 64, None, A, A, A, 1, None) == 2        # unsupported group
+    assert f(A, 1, 4, 128, 2, 128, None, A, A, None, 1, None) == 1    # null out
+    assert f(A, 1, 4, 128, 2, 128, None, None, A, A, 1, None) == 1    # null packed
+    assert f(A, 1, 4, 128, 2, 128, None, A, A, A + 2, 1, None) == 4   # misaligned out
+    assert f(A, 1, 4, 128, 2, 128, None, A, A + 2, A, 1, None) == 4   # misaligned norms
+    assert f(A, 1, 4, 128, 2, 128, A + 2, A, A, A, 1, None) == 4      # misaligned codebook
+    assert f(None, 1, 0, 128, 2, 128, None, None, None, None, 1, None) == 0  # empty
+    b = L.cq_fake_quantize_batch
+    good = (A, 4, 128, A, A, A)
+    p, _k = _fjobs(good, good)
+    assert b(p, -1, 1, 2, 128, None, 1, None) == 1
+    assert b(None, 1, 1, 2, 128, None, 1, None) == 1
+    assert b(p, 2, 1, 2, 128, None, 3, None) == 1                     # bad out dtype
+    assert b(p, 2, 0, 1, 128, None, 1, None) == 1                     # bits 1
+    p, _k = _fjobs(good, (A, 4, 128, A, A, None))
+    assert b(p, 2, 1, 2, 128, None, 1, None) == 1                     # second job: null out
+    p, _k = _fjobs(good, (A, 4, 128, A, A, A + 8))
+    assert b(p, 2, 1, 2, 128, None, 1, None) == 4                     # second job: misaligned out
+    p, _k = _fjobs((None, 0, 128, None, None, None), (None, 3, 0, None, None, None))
+    assert b(p, 2, 1, 4, 128, None, 0, None) == 0                     # only empty jobs
+    assert b(None, 0, 1, 2, 128, None, 1, None) == 0                  # nothing to do
 
 
 def test_binding_refuses_cpu_tensors(L):

@@ -452,6 +452,57 @@ def test_quantize_dequantize_indices_idempotent_and_norm_closed_form():
     assert np.array_equal(n2, want.astype(np.float16).view(np.uint16))
 
 
+# ----------------------------------------------------------------------------------------
+# fake quantisation (the pages' cq_quantize output)
+# ----------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [0, 2, 3, 4])
+def test_fake_quantize_spike_closed_form(bits):
+    """A group holding one value a at position p rotates to s_i |a| / sqrt(g) with
+    s_i = sign(a) (-1)^popcount(i & p), so every component picks C+ (the level nearest
+    +1/sqrt(g)) or C- (nearest -1/sqrt(g)).  Writing C_i = (C+ + C-)/2 + s_i (C+ - C-)/2 and
+    using the orthogonality of the Walsh rows, the inverse rotation is
+        w_hat = n16 sqrt(g) [ sign(a) (C+ - C-)/2 e_p + (C+ + C-)/2 e_0 ],
+    n16 = fp16(|a|).  A dropped term, a wrong sign, index or scale fails it."""
+    g = G128
+    cb = oracle.codebook(bits, g).astype(np.float64)
+    cp = cb[np.argmin(np.abs(cb - 1 / math.sqrt(g)))]
+    cm = cb[np.argmin(np.abs(cb + 1 / math.sqrt(g)))]
+    for p in (0, 1, 77, 127):
+        for a in (0.37, -2.5):
+            w = np.zeros((1, 2 * g))
+            w[0, g + p] = a  # second group; the first stays zero
+            got = oracle.fake_quantize(w, bits, g)
+            n16 = float(np.float16(abs(a)))
+            want = np.zeros(2 * g)
+            want[g + p] += n16 * math.sqrt(g) * math.copysign(1.0, a) * (cp - cm) / 2
+            want[g] += n16 * math.sqrt(g) * (cp + cm) / 2
+            assert np.allclose(got[0], want, rtol=1e-12, atol=1e-15), (bits, p, a)
+
+
+@pytest.mark.parametrize("bits", [0, 2, 3, 4])
+def test_fake_quantize_relative_mse_matches_sphere_closed_form(bits):
+    rng = np.random.default_rng(31)
+    w = rng.standard_normal((1024, 1024)) * 0.02
+    got = oracle.rel_mse(w, oracle.fake_quantize(w, bits))
+    want = expected_rel_mse(oracle.codebook(bits).astype(np.float64) * math.sqrt(128), 128)
+    assert abs(got - want) / want < 0.015
+
+
+def test_fake_quantize_zero_and_ragged_groups():
+    """Zero groups stay zero, and a ragged last group equals the zero-padded computation
+    with the padding columns dropped."""
+    rng = np.random.default_rng(32)
+    w = rng.standard_normal((5, 300)) * 0.02
+    w[2, :] = 0.0
+    pad = np.zeros((5, 384))
+    pad[:, :300] = w
+    for bits in (0, 2, 4):
+        got = oracle.fake_quantize(w, bits)
+        assert np.all(got[2] == 0.0)
+        assert np.array_equal(got, oracle.fake_quantize(pad, bits)[:, :300])
+
+
 def test_unpack_index_matches_numpy_fields():
     rng = np.random.default_rng(22)
     for bits in (2, 3, 4):

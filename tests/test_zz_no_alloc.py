@@ -37,7 +37,8 @@ def _static_call(packed, norms, rows, cols, bits, x, y, stream):
 
 
 @pytest.mark.parametrize("rows,cols,bits,batch", [(11008, 4096, 2, 1), (4096, 11008, 2, 8),
-                                                  (300, 1000, 3, 3), (64, 32768, 4, 2)])
+                                                  (300, 1000, 3, 3), (64, 32768, 4, 2),
+                                                  (300, 1000, 2, 20)])
 def test_static_scratch_gemv_matches_workspace_gemv_twice(rows, cols, bits, batch):
     dev = torch.device("cuda:0")
     w = torch.empty((rows, cols), dtype=torch.bfloat16, device=dev)
@@ -54,12 +55,18 @@ def test_static_scratch_gemv_matches_workspace_gemv_twice(rows, cols, bits, batc
         outs.append(y)
     torch.cuda.synchronize()
     r = ref.cpu().numpy().astype(np.float64)
+    # Up to 8 activation rows both entry points launch the same kernels with the same split:
+    # identical bits.  Above 8 the static one runs its blocks one launch pair at a time, so
+    # its split-K (chosen per launch) and hence the fp32 summation order may differ.
+    same_bits = batch <= 8
     for y in outs:
         parity.check_gemv(y.cpu().numpy(), r, "static scratch")
-        assert torch.equal(y, ref)  # same kernels, same order: identical bits
+        assert torch.equal(y, outs[0])
+        if same_bits:
+            assert torch.equal(y, ref)
     y3 = cq.dequant_gemv_static(packed, norms, rows, cols, bits, x)
     torch.cuda.synchronize()
-    assert torch.equal(y3, ref)
+    assert torch.equal(y3, outs[0])
 
 
 def test_static_scratch_rejects_columns_beyond_its_size():
