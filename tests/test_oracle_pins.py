@@ -153,8 +153,10 @@ def test_lloyd_max_with_page_parameters_near_closed_form(L, tol_level, tol_mse):
     assert abs(mse - ref_mse) / ref_mse < tol_mse
 
 
-def test_lloyd_max_two_bit_matches_printed_levels():
-    # benchmark spec prints the 2-bit Gaussian Lloyd-Max levels +-0.4528 / +-1.5104, MSE ~0.1175
+def test_lloyd_max_two_bit_matches_textbook_levels():
+    # The classical optimum 4-level quantiser of a unit Gaussian (J. Max, "Quantizing for
+    # minimum distortion", IRE Trans. Inf. Theory, 1960) has levels +-0.4528 / +-1.510 and
+    # mean squared error 0.1175.
     c = oracle.lloyd_max(4)
     assert np.allclose(np.abs(c), [1.5104, 0.4528, 0.4528, 1.5104], atol=5e-3)
     _, mse = gauss_lloyd_closed(4)
