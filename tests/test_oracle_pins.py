@@ -349,6 +349,15 @@ def test_quantize_bf16_input_reads_top_half_of_fp32():
     assert all(np.array_equal(x, y) for x, y in zip(oracle.quantize(bf, 2), oracle.quantize(exact, 2)))
 
 
+def test_fake_quantize_bf16_input_reads_top_half_of_fp32():
+    rng = np.random.default_rng(9)
+    w32 = (rng.standard_normal((3, 300)) * 0.02).astype(np.float32)
+    bf = (w32.view(np.uint32) >> 16).astype(np.uint16)
+    exact = (bf.astype(np.uint32) << 16).view(np.float32)
+    for bits in (0, 3):
+        assert np.array_equal(oracle.fake_quantize(bf, bits), oracle.fake_quantize(exact, bits))
+
+
 def test_norm_is_rotation_invariant():
     rng = np.random.default_rng(9)
     w = rng.standard_normal((64, 512)) * 0.02
@@ -517,7 +526,7 @@ def test_unpack_index_matches_numpy_fields():
 # GEMV
 # ----------------------------------------------------------------------------------------
 
-@pytest.mark.parametrize("rows,cols,batch", [(37, 300, 1), (16, 512, 8)])
+@pytest.mark.parametrize("rows,cols,batch", [(37, 300, 1), (16, 512, 8), (9, 260, 20)])
 def test_gemv_matches_hadamard_domain_identity(rows, cols, batch):
     rng = np.random.default_rng(rows + cols)
     w = rng.standard_normal((rows, cols)) * 0.02
