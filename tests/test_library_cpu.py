@@ -262,3 +262,12 @@ def test_binding_refuses_cpu_tensors(L):
     torch = pytest.importorskip("torch")
     with pytest.raises(ValueError):
         cq.quantize(torch.zeros(4, 128, dtype=torch.bfloat16), 2)
+    with pytest.raises(ValueError):
+        cq.fake_quantize(torch.zeros(4, 128, dtype=torch.bfloat16), 2)
+    with pytest.raises(ValueError):
+        cq.fake_quantize(torch.zeros(4, 128, dtype=torch.float16), 2)  # unsupported dtype
+    with pytest.raises(ValueError):
+        cq.fake_quantize_batch([torch.zeros(4, 128, dtype=torch.bfloat16)], 2)
+    with pytest.raises(ValueError):
+        cq.fake_quantize_batch([torch.zeros(4, 128, dtype=torch.bfloat16)], 2,
+                               outs=[torch.zeros(4, 64, dtype=torch.bfloat16)])  # shape mismatch
