@@ -63,3 +63,25 @@ def test_clock_sampler_parses_nvidia_smi_lines():
                "garbage"]
     s = c.summary()
     assert s["sm_mhz"] == 1882.5 and s["sm_max_mhz"] == 1965 and s["reasons"] == ["sw_power_cap"]
+
+
+def test_load_traffic_scales_per_weight_and_checks_the_source_hash(monkeypatch):
+    import json
+    from hadamard_codebook_bit_b200 import build as cq_build
+    with open(os.path.join(os.path.dirname(bench.__file__), "profiles", "traffic.json")) as f:
+        table = json.load(f)
+    n = 6_476_005_376
+    for kernel in ("quantize", "dequantize", "dequant_gemv"):
+        ent = table[kernel]
+        assert abs(ent["dram_bytes_per_weight"] - (ent["dram_read_bytes"] + ent["dram_write_bytes"]) / 134217728) < 1e-4
+        monkeypatch.setattr(cq_build, "source_hash", lambda h=ent["source_hash"]: h)
+        assert bench.load_traffic(kernel, n) == round(ent["dram_bytes_per_weight"] * n)
+    monkeypatch.setattr(cq_build, "source_hash", lambda: "0" * 16)  # kernels changed since capture
+    assert bench.load_traffic("dequantize", n) is None
+    assert bench.load_traffic("no_such_kernel", n) is None
+
+
+def test_arm_config_names_the_workload():
+    c1, c4 = bench.arm_config(1), bench.arm_config(4)
+    assert "6,476,005,376 weights" in c1["workload"] and c1["bits"] == 2 and c1["group_size"] == 128
+    assert c1["parallelism"] != c4["parallelism"] and "4" in c4["parallelism"]
