@@ -10,8 +10,9 @@ batch-1 product through every tensor.  Inputs are far larger than L2 (13 GB), so
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cq|reference]
 
 `value` is Gweights/s through the step (all ranks; weak scaling: each rank runs its own
-replica of the set).  Per-op times, 4-bit quantise / dequantise and the GEMV-only
-workload (the two MLP shapes over 48 distinct replicas, batch 1 and 8) are reported in
+replica of the set).  Per-op times, the same ops as one call per tensor, fake quantisation
+(bf16 -> bf16 through the stored form), 4-bit quantise / dequantise and the GEMV-only
+workload (the two MLP shapes over 48 distinct replicas, batch 1, 8 and 64) are reported in
 `breakdown`.  `--impl reference` times the CPU oracle on a bounded sample instead.
 """
 from __future__ import annotations
