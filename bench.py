@@ -562,17 +562,18 @@ def run_cuda_arm(args):
 
 def load_traffic(kernel: str, n_weights: int):
     """DRAM bytes per launch-unit from the committed ncu summary, scaled to this launch, or
-    None if the summary is missing or was taken on a different kernel source."""
+    None if the summary is missing or was taken on a different source of that kernel (its
+    .cu file and the headers it includes)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
         ent = d[kernel]
         from hadamard_codebook_bit_b200 import build as b
-        if ent.get("source_hash") != b.source_hash():
+        if ent.get("source_hash") != b.source_hash(ent.get("sources")):
             return None
         return round(ent["dram_bytes_per_weight"] * n_weights)
-    except (OSError, KeyError, ValueError, AttributeError):
+    except (OSError, KeyError, ValueError, AttributeError, FileNotFoundError):
         return None
 
 

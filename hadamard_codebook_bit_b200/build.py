@@ -41,11 +41,19 @@ def _deps() -> list[str]:
     return out
 
 
-def source_hash() -> str:
-    """SHA-256 over the kernel sources and the public header (identifies a kernel build)."""
+def source_hash(files=None) -> str:
+    """SHA-256 over the kernel sources and the public header (identifies a kernel build), or
+    over the named files only (base names under csrc/ or include/: one kernel and the headers
+    it includes)."""
     import hashlib
     h = hashlib.sha256()
-    for path in sorted(_deps()):
+    paths = _deps()
+    if files is not None:
+        want = set(files)
+        paths = [p for p in paths if os.path.basename(p) in want]
+        if {os.path.basename(p) for p in paths} != want:
+            raise FileNotFoundError(f"unknown sources: {sorted(want - {os.path.basename(p) for p in paths})}")
+    for path in sorted(paths):
         h.update(os.path.basename(path).encode())
         with open(path, "rb") as f:
             h.update(f.read())

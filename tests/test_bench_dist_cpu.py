@@ -74,9 +74,9 @@ def test_load_traffic_scales_per_weight_and_checks_the_source_hash(monkeypatch):
     for kernel in ("quantize", "dequantize", "dequant_gemv"):
         ent = table[kernel]
         assert abs(ent["dram_bytes_per_weight"] - (ent["dram_read_bytes"] + ent["dram_write_bytes"]) / 134217728) < 1e-4
-        monkeypatch.setattr(cq_build, "source_hash", lambda h=ent["source_hash"]: h)
+        monkeypatch.setattr(cq_build, "source_hash", lambda files=None, h=ent["source_hash"]: h)
         assert bench.load_traffic(kernel, n) == round(ent["dram_bytes_per_weight"] * n)
-    monkeypatch.setattr(cq_build, "source_hash", lambda: "0" * 16)  # kernels changed since capture
+    monkeypatch.setattr(cq_build, "source_hash", lambda files=None: "0" * 16)  # kernel changed since capture
     assert bench.load_traffic("dequantize", n) is None
     assert bench.load_traffic("no_such_kernel", n) is None
 
@@ -85,3 +85,12 @@ def test_arm_config_names_the_workload():
     c1, c4 = bench.arm_config(1), bench.arm_config(4)
     assert "6,476,005,376 weights" in c1["workload"] and c1["bits"] == 2 and c1["group_size"] == 128
     assert c1["parallelism"] != c4["parallelism"] and "4" in c4["parallelism"]
+
+
+def test_source_hash_of_named_files():
+    from hadamard_codebook_bit_b200 import build as cq_build
+    a = cq_build.source_hash(["cq_gemv.cu", "cq.h"])
+    assert a == cq_build.source_hash(["cq.h", "cq_gemv.cu"]) and a != cq_build.source_hash(["cq_gemv.cu"])
+    assert len(cq_build.source_hash()) == 16
+    with pytest.raises(FileNotFoundError):
+        cq_build.source_hash(["no_such_file.cu"])
