@@ -138,6 +138,39 @@ def _dev_ptr(t, name: str) -> int:
     return t.data_ptr()
 
 
+# The C ABI takes plain pointers and sizes, so a buffer smaller than a call touches would make
+# the kernels read or write past its end.  The binding checks every buffer first (dtype and
+# byte count: _fits, _check_stored, _check_x), then takes the pointers (_ptr: a contiguous
+# CUDA tensor on the call's device).
+
+def _fits(t, nbytes: int, name: str, dtype=None) -> None:
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}")
+    have = t.numel() * t.element_size()
+    if have < nbytes:
+        raise ValueError(f"{name} holds {have} bytes; the call needs {nbytes}")
+
+
+def _check_stored(packed, norms, rows: int, cols: int, bits: int, group_size: int) -> None:
+    torch = _torch()
+    _fits(packed, packed_bytes(rows, cols, bits, group_size), "packed", torch.uint8)
+    _fits(norms, norm_bytes(rows, cols, group_size), "norms", torch.float16)
+
+
+def _check_x(x, cols: int) -> None:
+    torch = _torch()
+    if x.dim() != 2 or x.shape[1] != cols:
+        raise ValueError(f"x must be [batch, {cols}]")
+    _fits(x, 0, "x", torch.bfloat16)
+
+
+def _ptr(t, name: str, device) -> int:
+    ptr = _dev_ptr(t, name)
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}")
+    return ptr
+
+
 def _cb_ptr(cb, device) -> int | None:
     if cb is None:
         return None
@@ -168,10 +201,11 @@ def quantize(w, bits: int, group_size: int = GROUP_SIZE, codebook=None, out=None
         raise ValueError("w must be bfloat16 or float32")
     rows, cols = w.shape
     packed, norms = out if out is not None else empty_packed(rows, cols, bits, w.device, group_size)
+    _check_stored(packed, norms, rows, cols, bits, group_size)
     with torch.cuda.device(w.device):
         _check(lib().cq_quantize(_dev_ptr(w, "w"), dt, rows, cols, bits, group_size,
-                                 _cb_ptr(codebook, w.device), _dev_ptr(packed, "packed"),
-                                 _dev_ptr(norms, "norms"), _stream(w.device)), "cq_quantize")
+                                 _cb_ptr(codebook, w.device), _ptr(packed, "packed", w.device),
+                                 _ptr(norms, "norms", w.device), _stream(w.device)), "cq_quantize")
     return packed, norms
 
 
@@ -198,6 +232,8 @@ def quantize_batch(ws, bits: int, group_size: int = GROUP_SIZE, codebook=None, o
         dt = CQ_F32
     else:
         raise ValueError("tensors must be bfloat16 or float32")
+    if outs is not None and len(outs) != len(ws):
+        raise ValueError("one (packed, norms) pair per tensor")
     jobs = (_QuantizeJob * len(ws))()
     res = []
     for k, w in enumerate(ws):
@@ -205,8 +241,8 @@ def quantize_batch(ws, bits: int, group_size: int = GROUP_SIZE, codebook=None, o
             raise ValueError("tensors must be 2-D, of one dtype, on one device")
         rows, cols = w.shape
         packed, norms = outs[k] if outs is not None else empty_packed(rows, cols, bits, dev, group_size)
-        jobs[k] = _QuantizeJob(_dev_ptr(w, "w"), rows, cols, _dev_ptr(packed, "packed"),
-                               _dev_ptr(norms, "norms"))
+        _check_stored(packed, norms, rows, cols, bits, group_size)
+        jobs[k] = _QuantizeJob(_dev_ptr(w, "w"), rows, cols, _ptr(packed, "packed", dev), _ptr(norms, "norms", dev))
         res.append((packed, norms))
     with torch.cuda.device(dev):
         _check(lib().cq_quantize_batch(ctypes.cast(jobs, ctypes.c_void_p), len(ws), dt, bits, group_size,
@@ -225,6 +261,8 @@ def dequantize_batch(items, bits: int, group_size: int = GROUP_SIZE, codebook=No
     if outs is None:
         out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
         outs = [torch.empty((r, c), dtype=out_dtype, device=dev) for _, _, r, c in items]
+    if len(outs) != len(items):
+        raise ValueError("one output per item")
     dtype = outs[0].dtype
     if dtype == torch.bfloat16:
         dt = CQ_BF16
@@ -234,12 +272,10 @@ def dequantize_batch(items, bits: int, group_size: int = GROUP_SIZE, codebook=No
         raise ValueError("out dtype must be bfloat16 or float32")
     jobs = (_DequantizeJob * len(items))()
     for k, ((packed, norms, rows, cols), out) in enumerate(zip(items, outs)):
-        if norms.dtype != torch.float16:
-            raise ValueError("norms must be float16")
-        if out.dtype != dtype or packed.device != dev or out.device != dev:
-            raise ValueError("outputs must share one dtype and device")
-        jobs[k] = _DequantizeJob(_dev_ptr(packed, "packed"), _dev_ptr(norms, "norms"), rows, cols,
-                                 _dev_ptr(out, "out"))
+        _check_stored(packed, norms, rows, cols, bits, group_size)
+        _fits(out, rows * cols * out.element_size(), "out", dtype)
+        jobs[k] = _DequantizeJob(_ptr(packed, "packed", dev), _ptr(norms, "norms", dev), rows, cols,
+                                 _ptr(out, "out", dev))
     with torch.cuda.device(dev):
         _check(lib().cq_dequantize_batch(ctypes.cast(jobs, ctypes.c_void_p), len(items), bits,
                                          group_size, _cb_ptr(codebook, dev), dt, _stream(dev)),
@@ -262,21 +298,24 @@ def dequant_gemv_batch(items, bits: int, group_size: int = GROUP_SIZE, codebook=
     if not items:
         return []
     dev = items[0][0].device
+    if (ys is not None and len(ys) != len(items)) or (workspaces is not None and len(workspaces) != len(items)):
+        raise ValueError("one y and one workspace per product")
     jobs = (_GemvJob * len(items))()
     out = []
     keep = []  # every job's workspace stays allocated until the launches are enqueued
     for k, (packed, norms, rows, cols, x) in enumerate(items):
         if x.dim() == 1:
             x = x.unsqueeze(0)
-        if x.dtype != torch.bfloat16 or norms.dtype != torch.float16:
-            raise ValueError("x must be bfloat16 and norms float16")
         batch = x.shape[0]
+        _check_x(x, cols)
+        _check_stored(packed, norms, rows, cols, bits, group_size)
         y = ys[k] if ys is not None else torch.empty((batch, rows), dtype=torch.float32, device=dev)
+        _fits(y, 4 * batch * rows, "y", torch.float32)
         wsb = gemv_workspace_bytes(cols, batch)
         ws = workspaces[k] if workspaces is not None else torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
         keep.append(ws)
-        jobs[k] = _GemvJob(_dev_ptr(packed, "packed"), _dev_ptr(norms, "norms"), rows, cols,
-                           _dev_ptr(x, "x"), batch, _dev_ptr(y, "y"), _dev_ptr(ws, "workspace"),
+        jobs[k] = _GemvJob(_ptr(packed, "packed", dev), _ptr(norms, "norms", dev), rows, cols,
+                           _ptr(x, "x", dev), batch, _ptr(y, "y", dev), _ptr(ws, "workspace", dev),
                            ws.numel() * ws.element_size())
         out.append(y)
     with torch.cuda.device(dev):
@@ -308,12 +347,16 @@ def fake_quantize(w, bits: int, group_size: int = GROUP_SIZE, codebook=None, out
     if out is None:
         out = torch.empty((rows, cols), dtype=w.dtype if out_dtype is None else out_dtype, device=w.device)
     ot = _dtype_code(out.dtype, "out")
+    if tuple(out.shape) != (rows, cols):
+        raise ValueError("out must have the shape of w")
     packed, norms = stored if stored is not None else empty_packed(rows, cols, bits, w.device, group_size)
-    with torch.cuda.device(w.device):
+    _check_stored(packed, norms, rows, cols, bits, group_size)
+    dev = w.device
+    with torch.cuda.device(dev):
         _check(lib().cq_fake_quantize(_dev_ptr(w, "w"), wt, rows, cols, bits, group_size,
-                                      _cb_ptr(codebook, w.device), _dev_ptr(packed, "packed"),
-                                      _dev_ptr(norms, "norms"), _dev_ptr(out, "out"), ot,
-                                      _stream(w.device)), "cq_fake_quantize")
+                                      _cb_ptr(codebook, dev), _ptr(packed, "packed", dev),
+                                      _ptr(norms, "norms", dev), _ptr(out, "out", dev), ot,
+                                      _stream(dev)), "cq_fake_quantize")
     return out
 
 
@@ -335,6 +378,8 @@ def fake_quantize_batch(ws, bits: int, group_size: int = GROUP_SIZE, codebook=No
     if outs is None:
         odt = ws[0].dtype if out_dtype is None else out_dtype
         outs = [torch.empty(tuple(w.shape), dtype=odt, device=dev) for w in ws]
+    if len(outs) != len(ws) or (stored is not None and len(stored) != len(ws)):
+        raise ValueError("one output (and one stored pair) per tensor")
     ot = _dtype_code(outs[0].dtype, "out")
     jobs = (_FakeQuantizeJob * len(ws))()
     keep = []  # intermediate buffers stay allocated until the launches are enqueued
@@ -346,8 +391,9 @@ def fake_quantize_batch(ws, bits: int, group_size: int = GROUP_SIZE, codebook=No
         rows, cols = w.shape
         packed, norms = stored[k] if stored is not None else empty_packed(rows, cols, bits, dev, group_size)
         keep.append((packed, norms))
-        jobs[k] = _FakeQuantizeJob(_dev_ptr(w, "w"), rows, cols, _dev_ptr(packed, "packed"),
-                                   _dev_ptr(norms, "norms"), _dev_ptr(out, "out"))
+        _check_stored(packed, norms, rows, cols, bits, group_size)
+        jobs[k] = _FakeQuantizeJob(_dev_ptr(w, "w"), rows, cols, _ptr(packed, "packed", dev),
+                                   _ptr(norms, "norms", dev), _ptr(out, "out", dev))
     with torch.cuda.device(dev):
         _check(lib().cq_fake_quantize_batch(ctypes.cast(jobs, ctypes.c_void_p), len(ws), wt, bits,
                                             group_size, _cb_ptr(codebook, dev), ot, _stream(dev)),
@@ -368,13 +414,13 @@ def dequantize(packed, norms, rows: int, cols: int, bits: int, group_size: int =
         dt = CQ_F32
     else:
         raise ValueError("out dtype must be bfloat16 or float32")
-    if norms.dtype != torch.float16:
-        raise ValueError("norms must be float16")
-    with torch.cuda.device(packed.device):
-        _check(lib().cq_dequantize(_dev_ptr(packed, "packed"), _dev_ptr(norms, "norms"), rows,
-                                   cols, bits, group_size, _cb_ptr(codebook, packed.device),
-                                   _dev_ptr(out, "out"), dt, _stream(packed.device)),
-               "cq_dequantize")
+    dev = packed.device
+    _check_stored(packed, norms, rows, cols, bits, group_size)
+    _fits(out, rows * cols * out.element_size(), "out")
+    with torch.cuda.device(dev):
+        _check(lib().cq_dequantize(_ptr(packed, "packed", dev), _ptr(norms, "norms", dev), rows, cols,
+                                   bits, group_size, _cb_ptr(codebook, dev), _ptr(out, "out", dev), dt,
+                                   _stream(dev)), "cq_dequantize")
     return out
 
 
@@ -387,20 +433,21 @@ def dequant_gemv(packed, norms, rows: int, cols: int, bits: int, x, group_size: 
     if x.dtype != torch.bfloat16:
         raise ValueError("x must be bfloat16")
     batch = x.shape[0]
-    if norms.dtype != torch.float16:
-        raise ValueError("norms must be float16")
+    dev = packed.device
+    _check_x(x, cols)
+    _check_stored(packed, norms, rows, cols, bits, group_size)
     if y is None:
-        y = torch.empty((batch, rows), dtype=torch.float32, device=packed.device)
+        y = torch.empty((batch, rows), dtype=torch.float32, device=dev)
+    _fits(y, 4 * batch * rows, "y", torch.float32)
     ws_bytes = gemv_workspace_bytes(cols, batch)
     if workspace is None:
-        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=packed.device)
-    with torch.cuda.device(packed.device):
-        _check(lib().cq_dequant_gemv(_dev_ptr(packed, "packed"), _dev_ptr(norms, "norms"), rows,
-                                     cols, bits, group_size, _cb_ptr(codebook, packed.device),
-                                     _dev_ptr(x, "x"), batch, _dev_ptr(y, "y"),
-                                     _dev_ptr(workspace, "workspace"),
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().cq_dequant_gemv(_ptr(packed, "packed", dev), _ptr(norms, "norms", dev), rows, cols,
+                                     bits, group_size, _cb_ptr(codebook, dev), _ptr(x, "x", dev), batch,
+                                     _ptr(y, "y", dev), _ptr(workspace, "workspace", dev),
                                      workspace.numel() * workspace.element_size(),
-                                     _stream(packed.device)), "cq_dequant_gemv")
+                                     _stream(dev)), "cq_dequant_gemv")
     return y
 
 
@@ -411,17 +458,16 @@ def dequant_gemv_static(packed, norms, rows: int, cols: int, bits: int, x,
     torch = _torch()
     if x.dim() == 1:
         x = x.unsqueeze(0)
-    if x.dtype != torch.bfloat16:
-        raise ValueError("x must be bfloat16")
-    if norms.dtype != torch.float16:
-        raise ValueError("norms must be float16")
     batch = x.shape[0]
+    dev = packed.device
+    _check_x(x, cols)
+    _check_stored(packed, norms, rows, cols, bits, group_size)
     if y is None:
-        y = torch.empty((batch, rows), dtype=torch.float32, device=packed.device)
-    with torch.cuda.device(packed.device):
-        _check(lib().cq_dequant_gemv_static(_dev_ptr(packed, "packed"), _dev_ptr(norms, "norms"),
-                                            rows, cols, bits, group_size,
-                                            _cb_ptr(codebook, packed.device), _dev_ptr(x, "x"),
-                                            batch, _dev_ptr(y, "y"), _stream(packed.device)),
-               "cq_dequant_gemv_static")
+        y = torch.empty((batch, rows), dtype=torch.float32, device=dev)
+    _fits(y, 4 * batch * rows, "y", torch.float32)
+    with torch.cuda.device(dev):
+        _check(lib().cq_dequant_gemv_static(_ptr(packed, "packed", dev), _ptr(norms, "norms", dev),
+                                            rows, cols, bits, group_size, _cb_ptr(codebook, dev),
+                                            _ptr(x, "x", dev), batch, _ptr(y, "y", dev),
+                                            _stream(dev)), "cq_dequant_gemv_static")
     return y

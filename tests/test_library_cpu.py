@@ -271,3 +271,117 @@ def test_binding_refuses_cpu_tensors(L):
     with pytest.raises(ValueError):
         cq.fake_quantize_batch([torch.zeros(4, 128, dtype=torch.bfloat16)], 2,
                                outs=[torch.zeros(4, 64, dtype=torch.bfloat16)])  # shape mismatch
+
+
+def test_binding_checks_buffer_sizes_before_any_call(L):
+    """The C ABI takes plain pointers, so the binding checks every buffer against the sizes
+    the call will touch (CPU tensors: the size checks come first, then 'must be a CUDA
+    tensor' for correctly sized ones)."""
+    torch = pytest.importorskip("torch")
+    rows, cols, bits = 4, 300, 2
+    G = 3
+    w = torch.zeros(rows, cols, dtype=torch.bfloat16)
+    ok_p = torch.zeros(rows, G, 32, dtype=torch.uint8)
+    ok_n = torch.zeros(rows, G, dtype=torch.float16)
+    small_p = torch.zeros(rows, G, 31, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="packed holds"):
+        cq.quantize(w, bits, out=(small_p, ok_n))
+    with pytest.raises(ValueError, match="norms must be"):
+        cq.quantize(w, bits, out=(ok_p, ok_n.view(torch.int16)))
+    with pytest.raises(ValueError, match="CUDA tensor|cuda device"):
+        cq.quantize(w, bits, out=(ok_p, ok_n))
+    with pytest.raises(ValueError, match="packed holds"):
+        cq.dequantize(small_p, ok_n, rows, cols, bits)
+    with pytest.raises(ValueError, match="out holds"):
+        cq.dequantize(ok_p, ok_n, rows, cols, bits, out=torch.zeros(rows, cols - 1, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="CUDA tensor|cuda device"):
+        cq.dequantize(ok_p, ok_n, rows, cols, bits, out=torch.zeros(rows, cols, dtype=torch.bfloat16))
+    x = torch.zeros(2, cols, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match=r"x must be \[batch, 300\]"):
+        cq.dequant_gemv(ok_p, ok_n, rows, cols, bits, torch.zeros(2, cols + 1, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="y holds"):
+        cq.dequant_gemv(ok_p, ok_n, rows, cols, bits, x, y=torch.zeros(2, rows - 1))
+    with pytest.raises(ValueError, match="CUDA tensor|cuda device"):
+        cq.dequant_gemv(ok_p, ok_n, rows, cols, bits, x, y=torch.zeros(2, rows))
+    with pytest.raises(ValueError, match="y holds"):
+        cq.dequant_gemv_static(ok_p, ok_n, rows, cols, bits, x, y=torch.zeros(1, rows))
+    with pytest.raises(ValueError, match="norms holds"):
+        cq.dequant_gemv_batch([(ok_p, ok_n[:, :2].contiguous(), rows, cols, x)], bits)
+    with pytest.raises(ValueError, match="one y and one workspace"):
+        cq.dequant_gemv_batch([(ok_p, ok_n, rows, cols, x)], bits, ys=[])
+    with pytest.raises(ValueError, match="one output per item"):
+        cq.dequantize_batch([(ok_p, ok_n, rows, cols)], bits, outs=[])
+    with pytest.raises(ValueError, match="one .packed, norms. pair per tensor"):
+        cq.quantize_batch([w, w], bits, outs=[(ok_p, ok_n)])
+    with pytest.raises(ValueError, match="packed holds"):
+        cq.fake_quantize(w, bits, stored=(small_p, ok_n))
+    with pytest.raises(ValueError, match="one output"):
+        cq.fake_quantize_batch([w, w], bits, outs=[w])
+
+
+class _FakeLib:
+    """Stands in for libcq in the marshalling test: records each call, launches nothing."""
+
+    def __init__(self, real):
+        self.real = real
+        self.calls = []
+
+    def __getattr__(self, name):
+        if name in ("cq_packed_bytes", "cq_norm_bytes", "cq_gemv_workspace_bytes", "cq_status_string"):
+            return getattr(self.real, name)
+
+        def call(*args):
+            self.calls.append((name, args))
+            return 0
+        return call
+
+
+def test_binding_marshals_valid_calls(L, monkeypatch):
+    """Every binding entry point accepts the shapes the GPU tests and the bench use (CPU
+    tensors stand in for device ones; the fake library records the calls)."""
+    torch = pytest.importorskip("torch")
+    import contextlib
+    fake = _FakeLib(L)
+    monkeypatch.setattr(cq, "lib", lambda: fake)
+    monkeypatch.setattr(cq, "_dev_ptr", lambda t, name: t.data_ptr())
+    monkeypatch.setattr(cq, "_stream", lambda device: 0)
+    monkeypatch.setattr(torch.cuda, "device", lambda d: contextlib.nullcontext())
+    bf = torch.bfloat16
+    for rows, cols, bits in ((37, 1000, 2), (4, 128, 0), (3, 129, 3), (5, 8, 4), (0, 128, 2), (7, 0, 2)):
+        w = torch.zeros(rows, cols, dtype=bf)
+        packed, norms = cq.quantize(w, bits)
+        cq.quantize(w.float(), bits, out=(packed, norms))
+        cq.dequantize(packed, norms, rows, cols, bits)
+        cq.dequantize(packed, norms, rows, cols, bits, out=torch.zeros(rows, cols))
+        cq.fake_quantize(w, bits)
+        cq.fake_quantize(w, bits, out=w, stored=(packed, norms))
+        cq.fake_quantize(w, bits, out_dtype=torch.float32)
+        for batch in (1, 8, 9, 64):
+            x = torch.zeros(batch, cols, dtype=bf)
+            cq.dequant_gemv(packed, norms, rows, cols, bits, x)
+            cq.dequant_gemv(packed, norms, rows, cols, bits, x, y=torch.zeros(batch, rows),
+                            workspace=torch.zeros(cq.gemv_workspace_bytes(cols, batch) or 16, dtype=torch.uint8))
+            cq.dequant_gemv_static(packed, norms, rows, cols, bits, x)
+        cq.dequant_gemv(packed, norms, rows, cols, bits, torch.zeros(cols, dtype=bf))  # 1-D x
+    # batched calls, including views of one flat buffer as the bench lays the set out
+    shapes = [(64, 256), (11, 1000), (0, 128), (3, 11008)]
+    ws = [torch.zeros(r, c, dtype=bf) for r, c in shapes]
+    q = cq.quantize_batch(ws, 2)
+    flat_p = torch.zeros(sum(p.numel() for p, _ in q), dtype=torch.uint8)
+    flat_n = torch.zeros(sum(n.numel() for _, n in q), dtype=torch.float16)
+    views, op, on = [], 0, 0
+    for p, n in q:
+        views.append((flat_p[op:op + p.numel()].view(p.shape), flat_n[on:on + n.numel()].view(n.shape)))
+        op += p.numel()
+        on += n.numel()
+    cq.quantize_batch(ws, 2, outs=views)
+    items = [(p, n, r, c) for (p, n), (r, c) in zip(views, shapes)]
+    cq.dequantize_batch(items, 2)
+    cq.dequantize_batch(items, 2, outs=[torch.zeros(r, c) for r, c in shapes])
+    cq.dequant_gemv_batch([(p, n, r, c, torch.zeros(1 + k, c, dtype=bf)) for k, (p, n, r, c) in enumerate(items)], 2)
+    cq.fake_quantize_batch(ws, 2)
+    cq.fake_quantize_batch(ws, 2, outs=ws, stored=views)
+    names = {n for n, _ in fake.calls}
+    assert names == {"cq_quantize", "cq_dequantize", "cq_fake_quantize", "cq_dequant_gemv",
+                     "cq_dequant_gemv_static", "cq_quantize_batch", "cq_dequantize_batch",
+                     "cq_dequant_gemv_batch", "cq_fake_quantize_batch"}
