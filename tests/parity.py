@@ -136,3 +136,35 @@ def check_gemv(gpu_y, ora_y, what=""):
         assert rel <= GEMV_REL_L2, f"{what}: batch row {b} rel L2 {rel:.3g}"
     return float(max(np.linalg.norm(g[b] - o[b]) / max(np.linalg.norm(o[b]), 1e-30)
                      for b in range(o.shape[0])))
+
+
+# ------------------------------------------------------------------------------------------
+# guard bytes around output buffers (stands in for a memory checker: a kernel that writes past
+# either end of its output changes the margins)
+# ------------------------------------------------------------------------------------------
+
+GUARD_BYTES = 4096
+GUARD_FILL = 0xA5
+
+
+def guarded_empty(shape, dtype, device):
+    """(base, t): `t` of `shape` and `dtype` lies inside `base`, a 1-D allocation with
+    GUARD_BYTES of GUARD_FILL before and after it.  t starts GUARD_BYTES into base, so it keeps
+    base's 16-byte alignment."""
+    import torch
+    numel = 1
+    for d in shape:
+        numel *= int(d)
+    esz = torch.empty((), dtype=dtype).element_size()
+    g = GUARD_BYTES // esz
+    base = torch.empty(numel + 2 * g, dtype=dtype, device=device)
+    base.view(torch.uint8).fill_(GUARD_FILL)
+    return base, base[g:g + numel].view(tuple(shape))
+
+
+def guard_intact(base, t) -> bool:
+    """True when both margins of `base` around `t` still hold GUARD_FILL."""
+    import torch
+    b = base.view(torch.uint8)
+    n = t.numel() * t.element_size()
+    return bool((b[:GUARD_BYTES] == GUARD_FILL).all() and (b[GUARD_BYTES + n:] == GUARD_FILL).all())

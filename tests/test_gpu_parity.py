@@ -494,6 +494,75 @@ def test_gemv_batch_many_jobs(ora):
         parity.check_gemv(to_np(ys[k]), ref, f"gemv batch job {k}")
 
 
+# ------------------------------------------------------------------------------------------
+# guard bytes: no kernel writes outside its output buffers (memory checkers are not available
+# here, so every output sits between margins of a fixed byte pattern that must survive)
+# ------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [0, 2, 3, 4])
+@pytest.mark.parametrize("rows,cols,dtype", [(37, 1000, torch.bfloat16), (5, 129, torch.float32),
+                                             (130, 4096, torch.bfloat16), (1, 8, torch.bfloat16),
+                                             (3, 11008, torch.bfloat16), (9, 100, torch.bfloat16)])
+def test_outputs_stay_inside_their_buffers(bits, rows, cols, dtype):
+    w = dev_tensor(rows, cols, dtype, 50, cols + bits, 0.02)
+    ref_p, ref_n = cq.quantize(w, bits)
+    G = -(-cols // 128)
+    bp, gp = parity.guarded_empty((rows, G, 16 * parity.field_bits(bits)), torch.uint8, DEV)
+    bn, gn = parity.guarded_empty((rows, G), torch.float16, DEV)
+    cq.quantize(w, bits, out=(gp, gn))
+    torch.cuda.synchronize()
+    assert parity.guard_intact(bp, gp) and parity.guard_intact(bn, gn)
+    assert torch.equal(gp, ref_p) and torch.equal(gn.view(torch.int16), ref_n.view(torch.int16))
+    for out_dtype in (torch.bfloat16, torch.float32):
+        ref_o = cq.dequantize(ref_p, ref_n, rows, cols, bits, out_dtype=out_dtype)
+        bo, go = parity.guarded_empty((rows, cols), out_dtype, DEV)
+        cq.dequantize(ref_p, ref_n, rows, cols, bits, out=go)
+        bf, gf = parity.guarded_empty((rows, cols), out_dtype, DEV)
+        cq.fake_quantize(w, bits, out=gf)
+        torch.cuda.synchronize()
+        assert parity.guard_intact(bo, go) and parity.guard_intact(bf, gf)
+        assert torch.equal(_int_view(go), _int_view(ref_o)) and torch.equal(_int_view(gf), _int_view(ref_o))
+    for batch in (1, 8, 20):
+        x = dev_tensor(batch, cols, torch.bfloat16, 51, cols + batch, 1.0)
+        ref_y = cq.dequant_gemv(ref_p, ref_n, rows, cols, bits, x)
+        bw, gw = parity.guarded_empty((cq.gemv_workspace_bytes(cols, batch),), torch.uint8, DEV)
+        by, gy = parity.guarded_empty((batch, rows), torch.float32, DEV)
+        cq.dequant_gemv(ref_p, ref_n, rows, cols, bits, x, workspace=gw, y=gy)
+        torch.cuda.synchronize()
+        assert parity.guard_intact(bw, gw) and parity.guard_intact(by, gy)
+        assert torch.equal(gy, ref_y)
+
+
+@pytest.mark.parametrize("bits", [0, 2, 4])
+def test_batched_outputs_stay_inside_their_buffers(bits):
+    ws = [batch_tensor(r, c, torch.bfloat16, 52, k, 0.02) for k, (r, c) in enumerate(BATCH_SHAPES)]
+    fb = parity.field_bits(bits)
+    gq = [(parity.guarded_empty((r, -(-c // 128), 16 * fb), torch.uint8, DEV),
+           parity.guarded_empty((r, -(-c // 128)), torch.float16, DEV)) for r, c in BATCH_SHAPES]
+    cq.quantize_batch(ws, bits, outs=[(p[1], n[1]) for p, n in gq])
+    go = [parity.guarded_empty((r, c), torch.bfloat16, DEV) for r, c in BATCH_SHAPES]
+    cq.dequantize_batch([(p[1], n[1], r, c) for (p, n), (r, c) in zip(gq, BATCH_SHAPES)], bits,
+                        outs=[o[1] for o in go])
+    gf = [parity.guarded_empty((r, c), torch.float32, DEV) for r, c in BATCH_SHAPES]
+    cq.fake_quantize_batch(ws, bits, outs=[f[1] for f in gf])
+    items, gy, gw = [], [], []
+    for k, ((p, n), (r, c)) in enumerate(zip(gq, BATCH_SHAPES)):
+        b = 1 + k % 3
+        items.append((p[1], n[1], r, c, batch_tensor(b, c, torch.bfloat16, 53, k, 1.0)))
+        gy.append(parity.guarded_empty((b, r), torch.float32, DEV))
+        gw.append(parity.guarded_empty((max(cq.gemv_workspace_bytes(c, b), 16),), torch.uint8, DEV))
+    cq.dequant_gemv_batch(items, bits, workspaces=[w_[1] for w_ in gw], ys=[y[1] for y in gy])
+    torch.cuda.synchronize()
+    for (p, n), o, f, y, w_, x, (r, c) in zip(gq, go, gf, gy, gw, ws, BATCH_SHAPES):
+        for base, t in (p, n, o, f, y, w_):
+            assert parity.guard_intact(base, t), (r, c)
+        sp, sn = cq.quantize(x, bits)
+        assert torch.equal(p[1], sp) and torch.equal(n[1].view(torch.int16), sn.view(torch.int16))
+        assert torch.equal(o[1].view(torch.int16), cq.dequantize(sp, sn, r, c, bits).view(torch.int16))
+        assert torch.equal(f[1].view(torch.int32),
+                           cq.dequantize(sp, sn, r, c, bits, out_dtype=torch.float32).view(torch.int32))
+
+
 def test_zz_no_kernel_wait_gave_up():
     """Every bounded wait inside the tensor-core kernels completed during this module."""
     assert cq.device_status() == 0

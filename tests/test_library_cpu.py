@@ -385,3 +385,20 @@ def test_binding_marshals_valid_calls(L, monkeypatch):
     assert names == {"cq_quantize", "cq_dequantize", "cq_fake_quantize", "cq_dequant_gemv",
                      "cq_dequant_gemv_static", "cq_quantize_batch", "cq_dequantize_batch",
                      "cq_dequant_gemv_batch", "cq_fake_quantize_batch"}
+
+
+def test_guard_helpers_detect_writes_past_either_end():
+    torch = pytest.importorskip("torch")
+    from tests import parity
+    for dtype in (torch.uint8, torch.float16, torch.bfloat16, torch.float32):
+        base, t = parity.guarded_empty((5, 7), dtype, "cpu")
+        assert t.shape == (5, 7) and (t.data_ptr() - base.data_ptr()) == parity.GUARD_BYTES
+        t.zero_()
+        assert parity.guard_intact(base, t)
+        flat = base.view(torch.uint8)
+        n = t.numel() * t.element_size()
+        flat[parity.GUARD_BYTES + n] = 0  # one byte past the end
+        assert not parity.guard_intact(base, t)
+        flat[parity.GUARD_BYTES + n] = parity.GUARD_FILL
+        flat[parity.GUARD_BYTES - 1] = 0  # one byte before the start
+        assert not parity.guard_intact(base, t)
