@@ -6,6 +6,9 @@
 //     <w_hat_rj, x_j> = <H (n_rj c[idx_rj]), x_j> = n_rj <c[idx_rj], H x_j>.
 // Each activation group is rotated once; the packed weights are never expanded in memory.
 //
+// A job carries at most 8 activation rows (the MMA's N); larger batches, up to 64, arrive as
+// one job per block of 8 rows with its own workspace slice (cq_api.cu).
+//
 // Step 1 (rotate_x_kernel, one block per group j, one warp per batch column b < 8):
 //   x~_bj = H_int x_bj (zero for b >= batch), scaled by 2^-e_bj so its largest magnitude sits
 //   in [2^13, 2^14), and written in the register-fragment order of the tensor-core B operand:
@@ -55,7 +58,7 @@ __host__ __device__ inline size_t frag_bytes(long long G) { return static_cast<s
 __host__ __device__ inline size_t scale_bytes(long long G) { return static_cast<size_t>(G) * kBatchCols * sizeof(float); }
 
 struct CodeTable {
-    uint32_t lo, hi;      // low / high bytes of the fp16 codewords 0..3 (2-bit codes)
+    uint32_t lo, hi;      // codes 0..3: int8 bytes of Ch / Cl (2-bit codes), else low / high fp16 bytes
     float inv_scale;      // 2^-cs: the table holds fp16(c_k 2^cs)
     uint32_t pad;
     uint16_t h[16];       // fp16 codewords 0..15 (entries past L repeat the last level)
