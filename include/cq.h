@@ -37,8 +37,9 @@
  *             pointers may then be NULL) and the GEMV writes y = 0 (rows * batch zeros).
  *   Errors    Arguments are validated on the host before anything is launched; a bad
  *             argument returns an error and launches nothing.  A failed launch returns
- *             CQ_ERR_CUDA.  Kernels never trap and never wait: codes beyond the last level
- *             (ternary code 3) decode as the last level.
+ *             CQ_ERR_CUDA.  Kernels never trap: codes beyond the last level (ternary
+ *             code 3) decode as the last level, and every wait inside a kernel is bounded
+ *             (cq_device_status reports one that gave up).
  *   Threads   Calls may come from several host threads; each call uses the device that
  *             is current on the calling thread.
  */
