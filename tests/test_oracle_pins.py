@@ -574,3 +574,21 @@ def test_packed_bytes_formula_and_config_totals():
     nb = sum(oracle.norm_bytes(r, c) for r, c in shapes)
     assert (idx, nb, idx + nb) == (11206656, 700416, 11907072)
     assert sum(r * c for r, c in shapes) == 44808192
+
+
+def test_oracle_results_do_not_depend_on_its_thread_count():
+    """The oracle spreads independent groups over threads; every output is computed by one
+    thread in a fixed order, so 1 thread and many give identical bits."""
+    rng = np.random.default_rng(40)
+    w = rng.standard_normal((67, 1000)) * 0.02
+    x = rng.standard_normal((3, 1000))
+    for bits in (0, 2, 3, 4):
+        p1, n1 = oracle.quantize(w, bits, nthreads=1)
+        p8, n8 = oracle.quantize(w, bits, nthreads=8)
+        assert np.array_equal(p1, p8) and np.array_equal(n1, n8)
+        d1 = oracle.dequantize(p1, n1, 67, 1000, bits, nthreads=1)
+        d8 = oracle.dequantize(p1, n1, 67, 1000, bits, nthreads=8)
+        assert np.array_equal(d1, d8)
+        y1 = oracle.dequant_gemv(p1, n1, 67, 1000, bits, x, nthreads=1)
+        y8 = oracle.dequant_gemv(p1, n1, 67, 1000, bits, x, nthreads=8)
+        assert np.array_equal(y1, y8)
